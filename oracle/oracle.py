@@ -1,0 +1,235 @@
+"""Float64 CPU oracle for the Gemma 1-4 decoder self-attention forward.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The CUDA library never
+calls it and shares no code with it: this file imports numpy and nothing else.
+
+Every step is the plain definition, evaluated in float64 on the (exactly
+widened) bf16 input values, in the order the layer applies them:
+
+1. QK-norm (RMSNorm per head over head_dim) -- KerasFormers "Gemma 4", What
+   changed (plain-weight RMSNorm, no 1+w offset); Gemma 3's usual 1+w gain;
+   norm_eps 1e-6 from the "Gemma" API table; QK-norm itself from the Atlas
+   "Gemma 4" summary (RMSNorm pre/post-norm + QK-norm).
+2. Rotary embedding, dual bases (KerasFormers "Gemma 3", What changed: rope_theta
+   1e6 global / rope_local_theta 1e4 local) with Gemma 4's partial rotation
+   (KerasFormers "Gemma 4", What changed: only partial_rotary_factor of each
+   head is rotated, the rest passed through).
+3. Scaled logits with query_pre_attn_scalar (ZeroModels "Gemma 2", API table).
+4. tanh logit softcapping c*tanh(s/c) (ZeroModels "Gemma 2", "Logit
+   softcapping" bullet: a scaled tanh).
+5. Causal mask, optionally limited to a sliding window (ZeroModels "Gemma 2",
+   "Alternating attention" bullet; KerasFormers "Gemma 3" API sliding_window).
+6. Softmax over the visible keys and the weighted sum of values; with K=V the
+   values are the key tensor as given (KerasFormers "Gemma 4", What changed:
+   key and value projections tied).
+7. GQA/MQA head grouping: query head h reads kv head h // (H / Hkv)
+   (KerasFormers "Gemma" API num_kv_heads=1; ZeroModels "Gemma 2" GQA bullet).
+
+Readings taken where the pages are silent (each is listed in the design doc):
+scale = scalar**-0.5; softcap after scaling; norm before RoPE; V is the raw k
+when keys and values are tied; rotated dims are the first R = fraction*D dims,
+paired rotate-half (t, t+R/2) with angle pos * theta**(-2t/F), F = head_dim by
+default; the window keeps keys with i - j < W; the mask works on token indices
+and positions only drive RoPE.
+
+Parity unpinned (no page value fixes them): the frequency denominator F of
+partial RoPE, the rotate-half pairing, and the window off-by-one.  The tests
+pin the oracle's arithmetic to closed forms, invariants, brute force and a
+library routine; they cannot pin those conventions.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+NORM_NONE = 0
+NORM_ONE_PLUS_W = 1
+NORM_W = 2
+
+
+def _f64(x):
+    """bf16/fp32 torch tensor or numpy array -> float64 numpy (exact widening)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().float().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# --- step 1: RMSNorm -------------------------------------------------------
+
+def rms_norm(x, w, mode: int, eps: float):
+    """x / sqrt(mean(x^2) + eps) * g over the last axis.
+
+    g = 1 + w (Gemma's usual offset), w (Gemma 4's plain weight), or 1 when
+    ``mode`` is NORM_NONE (then this function is the identity and is skipped).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if mode == NORM_NONE:
+        return x
+    w = np.asarray(w, dtype=np.float64)
+    g = (1.0 + w) if mode == NORM_ONE_PLUS_W else w
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * g
+
+
+# --- step 2: rotary embedding ----------------------------------------------
+
+def rope_angles(pos, rot_dim: int, theta: float, freq_dim: int):
+    """angle[p, t] = pos[p] * theta**(-2t/F) for t < rot_dim/2 (float64)."""
+    pos = np.asarray(pos, dtype=np.float64)
+    t = np.arange(rot_dim // 2, dtype=np.float64)
+    inv_freq = theta ** (-2.0 * t / freq_dim)
+    return pos[..., None] * inv_freq
+
+
+def rope(x, pos, rot_dim: int, theta: float, freq_dim: int):
+    """Rotate-half RoPE on dims [0, rot_dim); dims [rot_dim, D) pass through.
+
+    x: [..., D] with pos broadcastable to x.shape[:-1].  For t < R/2, with
+    a = x[t], b = x[t+R/2]:  x'[t] = a cos - b sin,  x'[t+R/2] = b cos + a sin.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if rot_dim == 0:
+        return x.copy()
+    half = rot_dim // 2
+    ang = rope_angles(pos, rot_dim, theta, freq_dim)
+    c, s = np.cos(ang), np.sin(ang)
+    out = x.copy()
+    a = x[..., :half]
+    b = x[..., half:rot_dim]
+    out[..., :half] = a * c - b * s
+    out[..., half:rot_dim] = b * c + a * s
+    return out
+
+
+# --- steps 3-5: logits, softcap, mask ----------------------------------------
+
+def softcap(s, c: float):
+    """c * tanh(s / c); c <= 0 means no cap."""
+    s = np.asarray(s, dtype=np.float64)
+    if c <= 0:
+        return s
+    return c * np.tanh(s / c)
+
+
+def visible(i, j, window: int):
+    """Key index j is visible to query index i: j <= i and (W == 0 or i - j < W)."""
+    i = np.asarray(i)
+    j = np.asarray(j)
+    ok = j <= i
+    if window > 0:
+        ok = ok & (i - j < window)
+    return ok
+
+
+def _attend(qt, kt, vals, q_idx, k_idx, scale, cap, window):
+    """Softmax attention of transformed queries qt [R,D] over keys kt [N,D]."""
+    s = (qt @ kt.T) * scale
+    s = softcap(s, cap)
+    mask = visible(q_idx[:, None], k_idx[None, :], window)
+    s = np.where(mask, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p = p / np.sum(p, axis=1, keepdims=True)
+    return p @ vals
+
+
+def _layer_fields(cfg):
+    get = (lambda k: cfg[k]) if isinstance(cfg, dict) else (lambda k: getattr(cfg, k))
+    D = get("head_dim")
+    frac = get("rotary_fraction")
+    rot = int(round(frac * D))
+    fd = get("rope_freq_dim") or D
+    return dict(H=get("num_heads"), Hkv=get("num_kv_heads"), D=D, W=get("window"),
+                theta=get("rope_theta"), rot=rot, F=fd, cap=get("softcap"),
+                scale=float(get("scalar")) ** -0.5, k_eq_v=bool(get("k_eq_v")),
+                mode=get("qk_norm"), eps=get("norm_eps"))
+
+
+# --- the layer: prefill ------------------------------------------------------
+
+def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None):
+    """Self-attention forward over a whole prompt (float64).
+
+    q [B,S,H,D], k [B,S,Hkv,D], v [B,S,Hkv,D] or None when cfg.k_eq_v,
+    positions [B,S] (drive RoPE only).  ``rows`` optionally restricts the
+    output to those query indices (same for every b, h).  Returns [B,R,H,D].
+    """
+    f = _layer_fields(cfg)
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    pos = np.asarray(_f64(positions))
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    assert H == f["H"] and Hkv == f["Hkv"] and D == f["D"] and H % Hkv == 0
+    G = H // Hkv
+    vals_all = k if f["k_eq_v"] else v
+    assert vals_all is not None
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    out = np.zeros((B, len(rows), H, D))
+    k_idx = np.arange(S)
+    for b in range(B):
+        kt = rope(rms_norm(k[b], w_k, f["mode"], f["eps"]), pos[b][:, None],
+                  f["rot"], f["theta"], f["F"])                      # [S,Hkv,D]
+        qt = rope(rms_norm(q[b, rows], w_q, f["mode"], f["eps"]), pos[b, rows][:, None],
+                  f["rot"], f["theta"], f["F"])                      # [R,H,D]
+        for h in range(H):
+            kv = h // G
+            out[b, :, h] = _attend(qt[:, h], kt[:, kv], vals_all[b, :, kv], rows, k_idx,
+                                   f["scale"], f["cap"], f["W"])
+    return out
+
+
+# --- the layer: one decode step ----------------------------------------------
+
+def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, batches=None):
+    """One decode step (float64): query b at position L_b - 1 over cache rows [0, L_b).
+
+    q [B,H,D]; k_cache / v_cache [B,Lmax,Hkv,D] raw (un-normed, un-rotated)
+    keys and values, or a list of per-batch [L_b,Hkv,D] arrays; cached key j
+    sits at position j.  ``batches`` restricts the output to those batch rows.
+    Returns [len(batches),H,D].
+    """
+    f = _layer_fields(cfg)
+    q = _f64(q)
+    B, H, D = q.shape
+    G = H // f["Hkv"]
+    seq_lens = np.asarray(_f64(seq_lens)).astype(np.int64)
+    batches = range(B) if batches is None else list(batches)
+    out = np.zeros((len(batches), H, D))
+    for n, b in enumerate(batches):
+        L = int(seq_lens[b])
+        kc = _f64(k_cache[b])[:L]
+        vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:L]
+        pos_k = np.arange(L)
+        kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],
+                  f["rot"], f["theta"], f["F"])
+        qt = rope(rms_norm(q[b], w_q, f["mode"], f["eps"]), np.array([L - 1]),
+                  f["rot"], f["theta"], f["F"])                       # [H,D]
+        for h in range(H):
+            kv = h // G
+            out[n, h] = _attend(qt[h:h + 1], kt[:, kv], vc[:, kv], np.array([L - 1]), pos_k,
+                                f["scale"], f["cap"], f["W"])[0]
+    return out
+
+
+# --- split-KV merge (decode's two-stage form) ---------------------------------
+
+def lse_merge(parts):
+    """Merge per-chunk softmax partials (m, l, O) of one query row.
+
+    Each chunk c contributes m_c = max of its logits, l_c = sum exp(s - m_c),
+    O_c = sum exp(s - m_c) v.  The merged row is
+    sum_c e^(m_c - M) O_c / sum_c e^(m_c - M) l_c with M = max_c m_c.
+    """
+    M = max(m for m, _, _ in parts)
+    num = sum(np.exp(m - M) * o for m, _, o in parts)
+    den = sum(np.exp(m - M) * l for m, l, _ in parts)
+    return num / den
+
+
+def chunk_partial(s, vals):
+    """(m, l, O) of one chunk: logits s [n] (already capped and masked), values [n,D]."""
+    m = np.max(s)
+    p = np.exp(s - m)
+    return m, np.sum(p), p @ vals

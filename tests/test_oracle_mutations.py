@@ -1,0 +1,99 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch each.
+
+Every mutation edits the oracle's source text, builds a throw-away module from
+it, and swaps its functions into the ``oracle`` package for the duration of the
+test.  The listed pins must then fail (raise AssertionError).  Nothing here
+touches a GPU.
+"""
+import inspect
+import types
+
+import pytest
+
+import oracle
+import oracle.oracle as src_mod
+import test_oracle as T
+
+MUTATIONS = {
+    # name: (original text, replacement, pins that must fail)
+    "rope_rotates_backwards": (
+        "out[..., :half] = a * c - b * s", "out[..., :half] = a * c + b * s",
+        [T.test_rope_worked_example, T.test_rope_is_complex_rotation]),
+    "rope_interleaved_pairs": (
+        "a = x[..., :half]\n    b = x[..., half:rot_dim]",
+        "a = x[..., 0:rot_dim:2]\n    b = x[..., 1:rot_dim:2]",
+        [T.test_rope_worked_example]),
+    "rope_frequency_uses_t_not_2t": (
+        "theta ** (-2.0 * t / freq_dim)", "theta ** (-1.0 * t / freq_dim)",
+        [T.test_rope_worked_example, T.test_rope_is_complex_rotation]),
+    "norm_drops_one_plus": (
+        "g = (1.0 + w) if mode == NORM_ONE_PLUS_W else w", "g = w",
+        [T.test_rms_norm_worked_example]),
+    "norm_sum_not_mean": (
+        "ms = np.mean(x * x, axis=-1, keepdims=True)", "ms = np.sum(x * x, axis=-1, keepdims=True)",
+        [T.test_rms_norm_worked_example]),
+    "norm_eps_outside_root": (
+        "return x / np.sqrt(ms + eps) * g", "return x / (np.sqrt(ms) + eps) * g",
+        [T.test_rms_norm_worked_example]),
+    "window_off_by_one": (
+        "ok = ok & (i - j < window)", "ok = ok & (i - j <= window)",
+        [T.test_mask_window_limits, T.test_mask_future_and_past_independence]),
+    "scale_divides_by_scalar": (
+        "scale=float(get(\"scalar\")) ** -0.5", "scale=1.0 / float(get(\"scalar\"))",
+        [T.test_worked_three_tokens]),
+    "softcap_drops_c": (
+        "return c * np.tanh(s / c)", "return np.tanh(s / c)",
+        [T.test_softcap_closed_form]),
+    "gqa_heads_strided": (
+        "            kv = h // G\n            out[b, :, h]", "            kv = h % Hkv\n            out[b, :, h]",
+        [T.test_mqa_equals_replicated_gqa]),
+    "keqv_values_are_normed_keys": (
+        "vals_all = k if f[\"k_eq_v\"] else v",
+        "vals_all = rms_norm(k, w_k, f[\"mode\"], f[\"eps\"]) if f[\"k_eq_v\"] else v",
+        [T.test_k_eq_v_is_passing_v_equals_k]),
+    "decode_query_one_past": (
+        "np.array([L - 1]),\n                  f[\"rot\"]", "np.array([L]),\n                  f[\"rot\"]",
+        [T.test_decode_equals_last_prefill_row]),
+    "softmax_drops_normaliser": (
+        "p = p / np.sum(p, axis=1, keepdims=True)", "p = p",
+        [T.test_softmax_of_constant_values, T.test_worked_three_tokens]),
+}
+
+
+def _mutated_module(old, new):
+    text = inspect.getsource(src_mod)
+    assert text.count(old) == 1, old
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(text.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+def _call(pin):
+    params = inspect.signature(pin).parameters
+    if not params:
+        return pin()
+    # parametrised pins: run their first parametrisation
+    marks = [m for m in getattr(pin, "pytestmark", []) if m.name == "parametrize"]
+    for m in marks:
+        names = [n.strip() for n in m.args[0].split(",")]
+        for values in m.args[1]:
+            values = values if isinstance(values, tuple) else (values,)
+            pin(**dict(zip(names, values)))
+    return None
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistakes_are_caught(name, monkeypatch):
+    old, new, pins = MUTATIONS[name]
+    mut = _mutated_module(old, new)
+    for attr in oracle.__all__:
+        monkeypatch.setattr(oracle, attr, getattr(mut, attr))
+    for pin in pins:
+        with pytest.raises(AssertionError):
+            _call(pin)
+
+
+def test_unmutated_pins_pass():
+    for _, _, pins in MUTATIONS.values():
+        for pin in pins:
+            _call(pin)
