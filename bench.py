@@ -1,0 +1,511 @@
+#!/usr/bin/env python
+"""Benchmark of the Gemma self-attention forward (libgattn) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: the Gemma-1-2b-shaped global MQA prefill (batch 4, seq 2048,
+8 query heads, 1 KV head, head_dim 256, full causal, RoPE theta 1e4), metric
+"attention prefill TFLOP/s" on effective (visible-pair) FLOPs.  A step is one
+gattn_prefill call (key prologue + tensor-core attention kernel) on inputs
+already resident in HBM; L2 is flushed (256 MiB write) before every step and
+the flush is outside the per-step CUDA-event timing.  Decode workloads report
+KV GB/s on algorithmic bytes.
+
+Under torchrun (N>1) every rank runs its own replica of the workload on its own
+GPU (independent problems, no collective on the data path: weak scaling); the
+time is the maximum over ranks.  ``--impl reference`` times the float64 CPU
+oracle instead (rank 0 only), on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+PREFILL_WL = {
+    "gemma1_2b_mqa_b4_s2048": W.GEMMA1_MQA,
+    "gemma2_2b_local_s256": W.GEMMA2_LOCAL,
+    "gemma3_1b_local_w512_b2_s8192": W.GEMMA3_LOCAL,
+    "gemma3_1b_global_b2_s8192": W.GEMMA3_GLOBAL,
+    "gemma4_12b_global_keqv_s32768": W.GEMMA4_GLOBAL,
+}
+DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
+                                 W.GEMMA4_DECODE_GLOBAL_NORM)}
+HEADLINE = "gemma1_2b_mqa_b4_s2048"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---- work counts -------------------------------------------------------------------------
+
+def visible_pairs(S: int, window: int) -> int:
+    """Visible (query, key) pairs of one causal sequence of S tokens."""
+    if window <= 0 or window >= S:
+        return S * (S + 1) // 2
+    return window * (window + 1) // 2 + (S - window) * window
+
+
+def row_visible(i, window):
+    i = np.asarray(i, dtype=np.int64)
+    return i + 1 if window <= 0 else np.minimum(i + 1, window)
+
+
+def prefill_flops(wl: W.PrefillWorkload) -> float:
+    L = wl.layer
+    return 4.0 * L.head_dim * L.num_heads * wl.batch * visible_pairs(wl.seq, L.window)
+
+
+def decode_bytes(layer: W.Layer, seq_lens) -> float:
+    n = np.asarray(seq_lens, dtype=np.int64)
+    if layer.window > 0:
+        n = np.minimum(n, layer.window)
+    per_row = layer.num_kv_heads * layer.head_dim * 2
+    kv = n.sum() * per_row * (1 if layer.k_eq_v else 2)
+    qo = len(n) * layer.num_heads * layer.head_dim * 2 * 2
+    return float(kv + qo)
+
+
+# ---- environment helpers ---------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(self.rows)}
+
+
+def source_hash(*paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name: str, kernel_src):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel."""
+    p = os.path.join(ROOT, "profiles", f"{name}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != source_hash(*kernel_src):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---- distributed plumbing ---------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x: float, device) -> float:
+    """Maximum of a float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---- the two arms ---------------------------------------------------------------------------
+
+def make_prefill(wl, dev):
+    from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
+    d = W.prefill_inputs(wl)
+    layer = AttentionLayer(LayerSpec.of(wl.layer), wl.seq, d["w_q"], d["w_k"], device=dev)
+    host = {k: d[k].pin_memory() for k in ("q", "k", "v", "positions") if d[k] is not None}
+    devt = {k: t.to(dev) for k, t in host.items()}
+    out = torch.empty_like(devt["q"])
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    ws = layer.prefill_workspace(wl.batch, wl.seq, dev)
+
+    def step(src=devt):
+        layer.prefill(src["q"], src["k"], src.get("v"), src["positions"], out=out, workspace=ws)
+
+    return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
+                work=prefill_flops(wl), unit="TFLOP/s", scale=1e12,
+                metric="attention prefill TFLOP/s (effective FLOPs)", bound="tensor",
+                launches=2 if (wl.layer.rot_dim or wl.layer.qk_norm) else 1,
+                kernel_src=("gemma_family_decoder_b200/csrc/prefill.cu",
+                            "gemma_family_decoder_b200/csrc/kernels/common.cuh"),
+                oracle=lambda: d)
+
+
+def make_decode(wl, dev):
+    from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
+    dq = W.decode_inputs(wl)
+    L = wl.layer
+    lens = dq["seq_lens"]
+    shape = (wl.batch, wl.max_len, L.num_kv_heads, L.head_dim)
+    k = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    v = None if L.k_eq_v else torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    for b in range(wl.batch):
+        n = int(lens[b])
+        lo = 0 if L.window == 0 else max(0, n - L.window)
+        rows = W.decode_cache_rows(wl, b, n - lo, lo)
+        k[b, lo:n] = rows["k"].to(dev)
+        if v is not None:
+            v[b, lo:n] = rows["v"].to(dev)
+    layer = AttentionLayer(LayerSpec.of(L), wl.max_len, dq["w_q"], dq["w_k"], device=dev)
+    host = {"q": dq["q"].pin_memory(), "seq_lens": lens.pin_memory()}
+    devt = {"q": host["q"].to(dev), "seq_lens": host["seq_lens"].to(dev), "k": k, "v": v}
+    out = torch.empty_like(devt["q"])
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    ws = layer.decode_workspace(wl.batch, wl.max_len, dev)
+
+    def step(src=devt):
+        layer.decode(src["q"], devt["k"], devt["v"], src["seq_lens"], out=out, workspace=ws)
+
+    return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
+                work=decode_bytes(L, lens.numpy()), unit="GB/s", scale=1e9,
+                metric="decode KV GB/s (algorithmic bytes)", bound="hbm", launches=2,
+                kernel_src=("gemma_family_decoder_b200/csrc/prep_decode.cu",
+                            "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
+
+
+def run_ours(args, world, rank, local):
+    from gemma_family_decoder_b200 import check, set_profile_events
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    is_prefill = name in PREFILL_WL
+    wl = PREFILL_WL[name] if is_prefill else DECODE_WL[name]
+    R = make_prefill(wl, dev) if is_prefill else make_decode(wl, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        R["step"]()
+    torch.cuda.synchronize()
+    st = check(R["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        set_profile_events(ev[i][2], ev[i][3])
+        R["step"]()
+        ev[i][1].record(stream)
+    set_profile_events(None, None)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    sampler.stop()
+    st = check(R["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed steps")
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    kern_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = reduce_max(sum(step_ms), dev)
+
+    # end to end through the public call: pinned host inputs in, result out, every step
+    E = max(3, min(K, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = sum(t.numel() * t.element_size() for t in R["host"].values())
+    d2h = R["out"].numel() * R["out"].element_size()
+    scratch = {k: torch.empty_like(t, device=dev) for k, t in R["host"].items()}
+    for it in range(E + 2):
+        if it == 2:
+            barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+        for k2, t in R["host"].items():
+            scratch[k2].copy_(t, non_blocking=True)
+        R["step"](scratch if is_prefill else dict(scratch))
+        R["host_out"].copy_(R["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / E
+
+    peaks, peak_src = load_peaks()
+    unit, scale = R["unit"], R["scale"]
+    value = R["work"] * world * K / (total_ms / 1e3) / scale
+    kern_mean = statistics.mean(kern_ms)
+    achieved = R["work"] / (kern_mean / 1e3) / scale
+    if R["bound"] == "tensor":
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        peak_unit = "TFLOP/s"
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        peak_unit = "GB/s"
+    traffic = profiled_traffic(name, R["kernel_src"])
+    result = {
+        "metric": R["metric"], "value": round(value, 3), "unit": unit, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": name, "l2": "flushed before every step (256 MiB write), "
+                   "flush outside the per-step CUDA-event time", "parallelism": f"replicas{world}"},
+        "roofline": {"bound": R["bound"], "achieved": round(achieved, 3), "peak": peak,
+                     "unit": peak_unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if R['bound'] == 'tensor' else 'hbm_gbs copy'})",
+                     "kernel_ms": round(kern_mean, 5)},
+        "e2e": {"value": round(R["work"] * world / (e2e_ms / 1e3) / scale, 3), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": R["launches"] * K,
+        "clocks": sampler.summary(),
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(name, budget_s=args.cpu_budget)
+    return result
+
+
+# ---- the float64 oracle on the host cores ---------------------------------------------------------
+
+def _oracle_prefill_rows(wl, d, rows):
+    import oracle as O
+    O.attention_prefill(d["q"], d["k"], d["v"], d["positions"], wl.layer, w_q=d["w_q"],
+                        w_k=d["w_k"], rows=rows)
+
+
+def cpu_baseline(name, budget_s=15.0):
+    """The oracle timed on a strided sample of query rows (prefill) or batch rows (decode)."""
+    import oracle as O
+    if name in PREFILL_WL:
+        wl = PREFILL_WL[name]
+        d = W.prefill_inputs(wl)
+        S = wl.seq
+        pilot = np.arange(0, S, max(1, S // 8))
+        t0 = time.perf_counter()
+        _oracle_prefill_rows(wl, d, pilot)
+        per_row = (time.perf_counter() - t0) / len(pilot)
+        n = int(max(8, min(S, budget_s / max(per_row, 1e-6))))
+        rows = np.unique(np.linspace(0, S - 1, n).astype(np.int64))
+        t0 = time.perf_counter()
+        _oracle_prefill_rows(wl, d, rows)
+        dt = time.perf_counter() - t0
+        L = wl.layer
+        work = 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(rows, L.window).sum())
+        return {"value": round(work / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                "kind": "oracle",
+                "sample": f"{len(rows)} evenly spaced query rows of {S}, all {wl.batch} sequences and "
+                          f"{L.num_heads} heads ({dt:.1f} s, float64 numpy)"}
+    wl = DECODE_WL[name]
+    dq = W.decode_inputs(wl)
+    lens = dq["seq_lens"].numpy()
+    L = wl.layer
+    done, t0, ks, vs, firsts = [], time.perf_counter(), [], [], []
+    for b in range(wl.batch):
+        n = int(lens[b])
+        lo = 0 if L.window == 0 else max(0, n - L.window)
+        rows = W.decode_cache_rows(wl, b, n - lo, lo)
+        ks.append(rows["k"])
+        vs.append(rows["v"])
+        firsts.append(lo)
+    t0 = time.perf_counter()
+    for b in range(wl.batch):
+        O.attention_decode(dq["q"], ks, None if L.k_eq_v else vs, dq["seq_lens"], L, w_q=dq["w_q"],
+                           w_k=dq["w_k"], batches=[b], first_rows=firsts)
+        done.append(b)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    work = decode_bytes(L, lens[done])
+    return {"value": round(work / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(done)} of {wl.batch} batch rows ({dt:.1f} s, float64 numpy)"}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step is a bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    import oracle as O  # noqa: F401
+    name = args.workload
+    budget = float(os.environ.get("GATTN_REF_BUDGET_S", "120"))
+    n_steps = args.steps + args.warmup
+    if name in PREFILL_WL:
+        wl = PREFILL_WL[name]
+        d = W.prefill_inputs(wl)
+        S, L = wl.seq, wl.layer
+        t0 = time.perf_counter()
+        _oracle_prefill_rows(wl, d, np.array([S - 1]))
+        per_row = time.perf_counter() - t0
+        rows_per_step = int(max(1, min(S, budget / n_steps / max(per_row, 1e-6))))
+        rng = np.random.default_rng(0)
+        work, dt = 0.0, 0.0
+        for i in range(n_steps):
+            rows = np.sort(rng.choice(S, size=rows_per_step, replace=False))
+            t0 = time.perf_counter()
+            _oracle_prefill_rows(wl, d, rows)
+            el = time.perf_counter() - t0
+            if i >= args.warmup:
+                dt += el
+                work += 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(rows, L.window).sum())
+        value, unit = work / dt / 1e12, "TFLOP/s"
+        sample = f"{rows_per_step} random query rows of {S} per step, all sequences and heads"
+        metric = "attention prefill TFLOP/s (effective FLOPs)"
+    else:
+        wl = DECODE_WL[name]
+        dq = W.decode_inputs(wl)
+        lens = dq["seq_lens"].numpy()
+        L = wl.layer
+        work, dt = 0.0, 0.0
+        for i in range(n_steps):
+            b = i % wl.batch
+            n = int(lens[b])
+            lo = 0 if L.window == 0 else max(0, n - L.window)
+            rows = W.decode_cache_rows(wl, b, n - lo, lo)
+            ks = [rows["k"] if j == b else None for j in range(wl.batch)]
+            vs = [rows["v"] if j == b else None for j in range(wl.batch)]
+            fr = [lo if j == b else 0 for j in range(wl.batch)]
+            t0 = time.perf_counter()
+            O.attention_decode(dq["q"], ks, None if L.k_eq_v else vs, dq["seq_lens"], L,
+                               w_q=dq["w_q"], w_k=dq["w_k"], batches=[b], first_rows=fr)
+            el = time.perf_counter() - t0
+            if i >= args.warmup:
+                dt += el
+                work += decode_bytes(L, lens[b:b + 1])
+        value, unit = work / dt / 1e9, "GB/s"
+        sample = "one batch row per step, cycling over the batch"
+        metric = "decode KV GB/s (algorithmic bytes)"
+    cores = blas_threads()
+    return {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name},
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(PREFILL_WL) + sorted(DECODE_WL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks have no work
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    world, rank, local = dist_setup()
+    if world != args.gpus and rank == 0:
+        print(f"note: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,77 @@
+// Internal launcher interface between the C-ABI host code (gattn_api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gattn {
+
+// Fields shared by every kernel, resolved from gattn_cfg on the host.
+struct LayerArgs {
+  int H, Hkv, G, D;
+  int window;
+  int rot;             // rotated dims R (0, or a power of two multiple of 16, <= D)
+  int rope_max_pos;
+  const float2* rope_tab;  // [max_pos][R/2] (cos, sin)
+  float softcap;       // 0 = off
+  float scale_log2;    // scalar^-1/2 * log2(e)
+  float scale;         // scalar^-1/2
+  int qk_norm;         // 0 none, 1 (1+w), 2 w
+  float eps;
+  const float* q_norm_w;
+  const float* k_norm_w;
+  int k_eq_v;
+};
+
+// RoPE table: (cos, sin) of p * theta^(-2t/F) for p < max_pos, t < half.
+cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim, int max_pos,
+                              cudaStream_t s);
+
+// k~ = RoPE(RMSNorm(k)) for every (b, s, kv head) row, bf16 out, same layout.
+cudaError_t launch_kprep(const __nv_bfloat16* k, const int* positions, __nv_bfloat16* kt,
+                         int B, int S, const LayerArgs& la, uint32_t* status, cudaStream_t s);
+
+// Split-KV decode: partials (m, l, O) per (b, h, split) then the merge.
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const int* seq_lens;
+  __nv_bfloat16* out;
+  int B, max_len;
+  int nsplit, chunk;
+  float* part_o;   // [B][H][nsplit][D]
+  float* part_ml;  // [B][H][nsplit][2]
+  uint32_t* status;
+};
+void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk);
+cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
+cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
+
+// Prefill on tcgen05 tensor cores.
+struct PrefillArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* kt;  // transformed keys (or raw k when no transform applies)
+  const __nv_bfloat16* v;   // values (raw k when k_eq_v)
+  const int* positions;
+  __nv_bfloat16* out;
+  int B, S;
+  uint32_t* status;
+  uint64_t timeout_ns;
+};
+cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
+
+// Self-test: one CTA waits on an mbarrier nobody arrives on.
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t s);
+
+// Wait limit used by every launch (ns).
+uint64_t wait_timeout_ns();
+
+// TMA descriptor encoding through the driver entry point (no -lcuda needed).
+bool encode_tmap_bshd(CUtensorMap* map, const void* base, int B, int S, int Hkv, int D,
+                      int box_rows);
+
+}  // namespace gattn

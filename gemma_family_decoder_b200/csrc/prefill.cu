@@ -1,0 +1,466 @@
+// Prefill self-attention on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// One CTA computes a 128-query tile of one head (and, for head_dim 512, one
+// 256-wide half of the value dims).  Warp roles:
+//   warps 0-3  query prologue (QK-norm + RoPE fused into the Q tile load), then
+//              per KV tile: S from TMEM -> scale, softcap, causal/window mask,
+//              online softmax with lazy rescale -> P (bf16) into shared memory;
+//              finally O / l -> bf16 -> global.
+//   warp 4     TMA producer: transformed-key tiles and value tiles into a
+//              two-stage shared-memory ring.
+//   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM slot, then
+//              O += P V into the TMEM accumulator.
+// KV tiles entirely outside the causal window are never visited.
+//
+// Layer definition: KerasFormers "Gemma 4" (What changed: plain-weight RMSNorm,
+// partial rotation, K=V global layers), KerasFormers "Gemma 3" (What changed:
+// dual RoPE bases), ZeroModels "Gemma 2" (logit softcapping, alternating
+// sliding-window attention, query_pre_attn_scalar).
+#include <cuda_bf16.h>
+
+#include "gattn_internal.h"
+#include "kernels/common.cuh"
+
+namespace gattn {
+
+using bf16 = __nv_bfloat16;
+
+template <int D, int BN>
+struct PrefillShape {
+  static constexpr int BM = 128;
+  static constexpr int DV = 256;                 // value dims per CTA
+  static constexpr int NSTAGE = 2;
+  static constexpr int KSTAGES = D / 256;        // ring stages per key tile
+  static constexpr int SLAB_KV = BN * 128;       // one 64-dim TMA box of BN rows
+  static constexpr int STAGE = 4 * SLAB_KV;      // 256 dims x BN rows
+  static constexpr int SLAB128 = BM * 128;       // 64 dims x 128 rows
+  static constexpr int Q_BYTES = (D / 64) * SLAB128;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = Q_BYTES;
+  static constexpr int OFF_P = OFF_RING + NSTAGE * STAGE;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int NBAR = 2 * NSTAGE + 8;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
+  static constexpr uint32_t TM_O = 0;
+  static constexpr uint32_t TM_S0 = DV;
+  static constexpr uint32_t TM_S1 = DV + BN;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(TM_S1 + BN <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct PrefillKParams {
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  const bf16* q;
+  bf16* out;
+  const int* positions;
+  uint32_t* status;
+  uint64_t timeout_ns;
+  int B, S, nqt, dv_splits;
+  LayerArgs la;
+};
+
+template <int D, int BN>
+__global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ PrefillKParams P) {
+  using C = PrefillShape<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::NSTAGE;
+  uint64_t* s_full = bars + 2 * C::NSTAGE;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* q_ready = o_done + 1;
+  uint64_t* drain = q_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const LayerArgs& la = P.la;
+  const int H = la.H, S = P.S;
+  // work item: heaviest query tiles first
+  int idx = blockIdx.x;
+  const int per_qt = P.B * H * P.dv_splits;
+  const int qt = P.nqt - 1 - idx / per_qt;
+  idx %= per_qt;
+  const int dvs = idx % P.dv_splits;
+  idx /= P.dv_splits;
+  const int h = idx % H;
+  const int b = idx / H;
+  const int kvh = h / la.G;
+  const int q0 = qt * C::BM;
+  const int dv_lo = dvs * C::DV;
+  const int kv_hi = min(S, q0 + C::BM);
+  const int kv_lo = la.window > 0 ? max(0, q0 - la.window + 1) : 0;
+  const int k_first = (kv_lo / BN) * BN;
+  const int ntiles = (kv_hi - k_first + BN - 1) / BN;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(q_ready, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&P.tm_k);
+    tma_prefetch_desc(&P.tm_v);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = P.timeout_ns;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------------ softmax
+    const int t = threadIdx.x;
+    const int qi = q0 + t;
+    const bool valid = qi < S;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // query prologue: RMSNorm + RoPE in fp32, bf16 into the swizzled Q tile
+    {
+      uint8_t* qs = smem + C::OFF_Q;
+      const bf16* qrow = P.q + ((static_cast<size_t>(b) * S + qi) * H + h) * D;
+      int pos = 0;
+      float r = 1.f;
+      if (valid) {
+        if (la.rot > 0) {
+          pos = __ldg(P.positions + static_cast<size_t>(b) * S + qi);
+          if (pos < 0 || pos >= la.rope_max_pos) {
+            flag_status(P.status, kStatusBounds);
+            pos = pos < 0 ? 0 : la.rope_max_pos - 1;
+          }
+        }
+        if (la.qk_norm) {
+          float ss = 0.f;
+          for (int c = 0; c < D / 8; ++c) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow) + c);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = unpack_bf16x2(w[e]);
+              ss += f.x * f.x + f.y * f.y;
+            }
+          }
+          r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+        }
+      }
+      const float off = la.qk_norm == 1 ? 1.f : 0.f;
+      const int half = la.rot >> 1;
+      const float2* trow = la.rope_tab + static_cast<size_t>(pos) * (half > 0 ? half : 1);
+      auto load8 = [&](int c, float (&x)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow) + c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w[e]);
+          x[2 * e] = f.x;
+          x[2 * e + 1] = f.y;
+        }
+        if (la.qk_norm) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = x[e] * r * (__ldg(la.q_norm_w + 8 * c + e) + off);
+        }
+      };
+      auto store8 = [&](int c, const float (&x)[8]) {
+        uint4 u;
+        u.x = pack_bf16x2(x[0], x[1]);
+        u.y = pack_bf16x2(x[2], x[3]);
+        u.z = pack_bf16x2(x[4], x[5]);
+        u.w = pack_bf16x2(x[6], x[7]);
+        const int phys = (c & 7) ^ (t & 7);
+        *reinterpret_cast<uint4*>(qs + (c >> 3) * C::SLAB128 + t * 128 + phys * 16) = u;
+      };
+      for (int c = 0; c < D / 8; ++c) {
+        float x[8];
+        if (!valid) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = 0.f;
+          store8(c, x);
+        } else if (8 * c < la.rot) {
+          if (8 * c >= half) continue;  // written with its partner
+          const int cp = c + (half >> 3);
+          float y[8];
+          load8(c, x);
+          load8(cp, y);
+          float xo[8], yo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 cs = __ldg(trow + 8 * c + e);
+            xo[e] = x[e] * cs.x - y[e] * cs.y;
+            yo[e] = y[e] * cs.x + x[e] * cs.y;
+          }
+          store8(c, xo);
+          store8(cp, yo);
+        } else {
+          load8(c, x);
+          store8(c, x);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_ready);
+    }
+
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t scol = tmem + lane_off + ((j & 1) ? C::TM_S1 : C::TM_S0);
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(scol + c * 32, rr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[j & 1]);
+
+      const int key0 = k_first + j * BN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        float x;
+        if (la.softcap > 0.f) {
+          x = la.softcap * tanhf(s[c] * la.scale / la.softcap) * 1.4426950408889634f;
+        } else {
+          x = s[c] * la.scale_log2;
+        }
+        const int key = key0 + c;
+        const bool vis = valid && key <= qi && (la.window <= 0 || qi - key < la.window);
+        x = vis ? x : -INFINITY;
+        s[c] = x;
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m, mx);
+      float alpha = 1.f;
+      bool rescale = false;
+      float m_use = m;
+      if (m_new > m + 8.f) {
+        m_use = m_new;
+        rescale = (m != -INFINITY);
+        alpha = rescale ? ex2(m - m_new) : 0.f;
+      }
+      const float mu = (m_use == -INFINITY) ? 0.f : m_use;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        const float p = ex2(s[c] - mu);
+        s[c] = p;
+        rs += p;
+      }
+      if (j >= 1) {
+        if (!mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (rescale) {
+#pragma unroll 1
+          for (int c = 0; c < C::DV / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st32(tmem + lane_off + C::TM_O + c * 32, rr);
+          }
+          tmem_wait_st();
+        }
+      }
+      l = (rescale ? l * alpha : l) + rs;
+      if (m_use != m) m = m_use;
+      // P row t (keys contiguous, 128-byte swizzle), 64 keys per slab
+      uint8_t* ps = smem + C::OFF_P;
+#pragma unroll
+      for (int ch = 0; ch < BN / 8; ++ch) {
+        uint4 u;
+        u.x = pack_bf16x2(s[8 * ch + 0], s[8 * ch + 1]);
+        u.y = pack_bf16x2(s[8 * ch + 2], s[8 * ch + 3]);
+        u.z = pack_bf16x2(s[8 * ch + 4], s[8 * ch + 5]);
+        u.w = pack_bf16x2(s[8 * ch + 6], s[8 * ch + 7]);
+        const int phys = (ch & 7) ^ (t & 7);
+        *reinterpret_cast<uint4*>(ps + (ch >> 3) * C::SLAB128 + t * 128 + phys * 16) = u;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag)) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* orow = P.out + ((static_cast<size_t>(b) * S + qi) * H + h) * D + dv_lo;
+#pragma unroll 1
+      for (int c = 0; c < C::DV / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, rr);
+        tmem_wait_ld();
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
+            dst[v] = u;
+          }
+        }
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int n = 0;
+      auto load = [&](const CUtensorMap* tm, int d_base, int key0) -> bool {
+        const int st = n % C::NSTAGE;
+        const uint32_t par = ((n / C::NSTAGE) & 1) ^ 1;
+        if (!mbar_wait(&empty[st], par, tmo, P.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(&full[st], C::STAGE);
+        uint8_t* dst = smem + C::OFF_RING + st * C::STAGE;
+#pragma unroll
+        for (int sub = 0; sub < 4; ++sub)
+          tma_load_4d(dst + sub * C::SLAB_KV, tm, &full[st], d_base + sub * 64, kvh, key0, b);
+        ++n;
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int key0 = k_first + j * BN;
+        for (int ks = 0; ks < C::KSTAGES && ok; ++ks) ok = load(&P.tm_k, ks * 256, key0);
+        if (ok && j >= 1) ok = load(&P.tm_v, dv_lo, key0 - BN);
+      }
+      if (ok) load(&P.tm_v, dv_lo, k_first + (ntiles - 1) * BN);
+      // let every issued copy land before the CTA can exit
+      for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)
+        mbar_wait(&full[i % C::NSTAGE], (i / C::NSTAGE) & 1, tmo, P.status, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
+      int n = 0;
+      bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
+      tc_fence_after();
+      auto qk = [&](int j) -> bool {
+        const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
+        for (int ks = 0; ks < C::KSTAGES; ++ks) {
+          const int st = n % C::NSTAGE;
+          if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t kb = sbase + C::OFF_RING + st * C::STAGE;
+#pragma unroll
+          for (int kk = 0; kk < 16; ++kk) {
+            const int dim = ks * 256 + kk * 16;
+            const uint64_t a = smem_desc_sw128(
+                sbase + C::OFF_Q + (dim >> 6) * C::SLAB128 + (dim & 63) * 2, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * C::SLAB_KV + (kk & 3) * 32, 16, 1024);
+            mma_bf16_ss(s_tm, a, bd, idesc_qk, (ks | kk) != 0);
+          }
+          mma_commit(&empty[st]);
+          ++n;
+        }
+        mma_commit(&s_full[j & 1]);
+        return true;
+      };
+      auto pv = [&](int i) -> bool {
+        if (!mbar_wait(p_full, i & 1, tmo, P.status, abort_flag)) return false;
+        const int st = n % C::NSTAGE;
+        if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = sbase + C::OFF_RING + st * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = smem_desc_sw128(
+              sbase + C::OFF_P + (kk >> 2) * C::SLAB128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
+          mma_bf16_ss(tmem + C::TM_O, a, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[st]);
+        ++n;
+        mma_commit(o_done);
+        return true;
+      };
+      for (int j = 0; j < ntiles && ok; ++j) {
+        if (j >= 2) ok = mbar_wait(&s_empty[j & 1], ((j >> 1) - 1) & 1, tmo, P.status, abort_flag);
+        if (ok) ok = qk(j);
+        if (ok && j >= 1) ok = pv(j - 1);
+      }
+      if (ok) pv(ntiles - 1);
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, tmo, P.status, nullptr);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, int BN>
+static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+  using C = PrefillShape<D, BN>;
+  PrefillKParams P;
+  if (!encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN)) return cudaErrorInvalidValue;
+  if (!encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN)) return cudaErrorInvalidValue;
+  P.q = pa.q;
+  P.out = pa.out;
+  P.positions = pa.positions;
+  P.status = pa.status;
+  P.timeout_ns = pa.timeout_ns;
+  P.B = pa.B;
+  P.S = pa.S;
+  P.nqt = (pa.S + C::BM - 1) / C::BM;
+  P.dv_splits = D / C::DV;
+  P.la = la;
+  auto kern = prefill_kernel<D, BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const long long grid = static_cast<long long>(P.nqt) * pa.B * la.H * P.dv_splits;
+  kern<<<static_cast<unsigned>(grid), 192, C::SMEM, s>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+  if (la.D == 256) return run_prefill<256, 128>(pa, la, s);
+  if (la.D == 512) return run_prefill<512, 64>(pa, la, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gattn

@@ -1,0 +1,427 @@
+// RoPE table, key prologue (QK-norm + RoPE) and the split-KV decode kernels.
+//
+// Decode follows the layer definition of the Gemma model cards for one new
+// token: the query at position L-1 attends over cache rows [0, L) (the last
+// `window` of them on sliding-window layers), keys pass through QK-norm and
+// RoPE at their own positions, and with K=V the raw cached keys are the
+// values (KerasFormers "Gemma 4", What changed).  The cache read is split in
+// chunks across CTAs; each CTA writes a (max, sum, weighted-sum) partial and a
+// second kernel merges them with the log-sum-exp rule.
+#include <cuda_bf16.h>
+
+#include "gattn_internal.h"
+#include "kernels/common.cuh"
+
+namespace gattn {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------------------
+// RoPE table: tab[p][t] = (cos, sin)(p * theta^(-2t/F)), angle in double.
+// ---------------------------------------------------------------------------
+__global__ void rope_table_kernel(float2* tab, double theta, int half, int freq_dim,
+                                  long long total) {
+  long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i >= total) return;
+  const int p = static_cast<int>(i / half);
+  const int t = static_cast<int>(i % half);
+  const double inv_freq = pow(theta, -2.0 * t / static_cast<double>(freq_dim));
+  double sn, cs;
+  sincos(static_cast<double>(p) * inv_freq, &sn, &cs);
+  tab[i] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+}
+
+cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim, int max_pos,
+                              cudaStream_t s) {
+  const long long total = static_cast<long long>(max_pos) * half;
+  const int threads = 256;
+  const long long blocks = (total + threads - 1) / threads;
+  rope_table_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(tab, theta, half, freq_dim,
+                                                                      total);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Shared row helpers: a warp holds one head row, lane l owning dims
+// [8(l+32i), 8(l+32i)+8) for i < D/256.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int NCH>
+__device__ __forceinline__ void load_row(const bf16* row, int lane, float (&x)[NCH][8]) {
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + lane + 32 * i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(w[e]);
+      x[i][2 * e] = f.x;
+      x[i][2 * e + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ int checked_pos(int pos, const LayerArgs& la, uint32_t* status) {
+  if (pos < 0 || pos >= la.rope_max_pos) {
+    flag_status(status, kStatusBounds);
+    return pos < 0 ? 0 : la.rope_max_pos - 1;
+  }
+  return pos;
+}
+
+// RMSNorm (optional) then RoPE (optional) on a warp-held row, in fp32.
+template <int NCH>
+__device__ __forceinline__ void transform_row(float (&x)[NCH][8], int lane, int pos,
+                                              const LayerArgs& la, const float* w,
+                                              uint32_t* status) {
+  constexpr int D = NCH * 256;
+  if (la.qk_norm) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += x[i][e] * x[i][e];
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+    const float off = la.qk_norm == 1 ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int d = 8 * (lane + 32 * i) + e;
+        x[i][e] = x[i][e] * r * (__ldg(w + d) + off);
+      }
+  }
+  if (la.rot > 0) {
+    pos = checked_pos(pos, la, status);
+    const int half = la.rot >> 1;
+    const int h16 = la.rot >> 4;  // chunks in half the rotated slice
+    float pr[NCH][8];
+    if (h16 < 32) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = __shfl_xor_sync(0xffffffffu, x[i][e], h16);
+    } else {
+      // rotated slice of 512 dims: the partner chunk is this lane's other chunk
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = x[NCH - 1 - i][e];
+    }
+    const float2* trow = la.rope_tab + static_cast<size_t>(pos) * half;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = lane + 32 * i;
+      if (8 * c < la.rot) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int d = 8 * c + e;
+          const bool first = d < half;
+          const float2 cs = __ldg(trow + (first ? d : d - half));
+          x[i][e] = first ? x[i][e] * cs.x - pr[i][e] * cs.y : x[i][e] * cs.x + pr[i][e] * cs.y;
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Key prologue for prefill: one warp per (b, s, kv head) row.
+// ---------------------------------------------------------------------------
+template <int NCH>
+__global__ void __launch_bounds__(256) kprep_kernel(const bf16* __restrict__ k,
+                                                    const int* __restrict__ positions,
+                                                    bf16* __restrict__ kt, long long rows,
+                                                    LayerArgs la, uint32_t* status) {
+  constexpr int D = NCH * 256;
+  const int lane = threadIdx.x & 31;
+  const long long row = blockIdx.x * 8LL + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const long long bs = row / la.Hkv;
+  const int pos = positions ? __ldg(positions + bs) : 0;
+  float x[NCH][8];
+  load_row<NCH>(k + row * D, lane, x);
+  transform_row<NCH>(x, lane, pos, la, la.k_norm_w, status);
+  uint4* dst = reinterpret_cast<uint4*>(kt + row * D);
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    uint4 u;
+    u.x = pack_bf16x2(x[i][0], x[i][1]);
+    u.y = pack_bf16x2(x[i][2], x[i][3]);
+    u.z = pack_bf16x2(x[i][4], x[i][5]);
+    u.w = pack_bf16x2(x[i][6], x[i][7]);
+    dst[lane + 32 * i] = u;
+  }
+}
+
+cudaError_t launch_kprep(const bf16* k, const int* positions, bf16* kt, int B, int S,
+                         const LayerArgs& la, uint32_t* status, cudaStream_t s) {
+  const long long rows = static_cast<long long>(B) * S * la.Hkv;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  if (la.D == 256)
+    kprep_kernel<1><<<blocks, 256, 0, s>>>(k, positions, kt, rows, la, status);
+  else
+    kprep_kernel<2><<<blocks, 256, 0, s>>>(k, positions, kt, rows, la, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV decode.  CTA = (split, kv head, b); NW warps.  Warp w serves the
+// head group hg = w % NHG (HPW query heads) and the key lane kg = w / NHG,
+// striding over the chunk's keys by KW = NW / NHG.
+// ---------------------------------------------------------------------------
+constexpr int kDecodeWarps = 4;
+
+template <int NCH, int HPW>
+__global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(DecodeArgs da,
+                                                                          LayerArgs la) {
+  constexpr int D = NCH * 256;
+  constexpr int NW = kDecodeWarps;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = la.G;
+  const int NHG = G / HPW;
+  const int KW = NW / NHG;
+  extern __shared__ float smem[];
+  float* qt = smem;                 // [G][D]
+  float* pm = qt + G * D;           // [NW][HPW]
+  float* pl = pm + NW * HPW;        // [NW][HPW]
+  float* po = pl + NW * HPW;        // [NW][HPW][D]
+
+  const size_t head0 = static_cast<size_t>(b) * la.H + static_cast<size_t>(kvh) * G;
+  const int L = __ldg(da.seq_lens + b);
+  const int lo = (L >= 1 && la.window > 0) ? max(0, L - la.window) : 0;
+  const int start = lo + split * da.chunk;
+  const int end = min(L, start + da.chunk);
+  if (L < 1 || L > da.max_len || start >= end) {
+    if (L < 1 || L > da.max_len) {
+      if (threadIdx.x == 0 && split == 0 && kvh == 0) flag_status(da.status, kStatusBounds);
+    }
+    for (int h = threadIdx.x; h < G; h += blockDim.x) {
+      float* ml = da.part_ml + ((head0 + h) * da.nsplit + split) * 2;
+      ml[0] = -INFINITY;
+      ml[1] = 0.f;
+    }
+    return;
+  }
+
+  // query prologue: norm, rope at position L-1, fold scale*log2(e)
+  for (int h = warp; h < G; h += NW) {
+    float x[NCH][8];
+    load_row<NCH>(da.q + (head0 + h) * D, lane, x);
+    transform_row<NCH>(x, lane, L - 1, la, la.q_norm_w, da.status);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qt[h * D + 8 * (lane + 32 * i) + e] = x[i][e] * la.scale_log2;
+  }
+  __syncthreads();
+
+  const int hg = warp % NHG, kg = warp / NHG;
+  float qreg[HPW][NCH][8];
+#pragma unroll
+  for (int hh = 0; hh < HPW; ++hh)
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qreg[hh][i][e] = qt[(hg * HPW + hh) * D + 8 * (lane + 32 * i) + e];
+
+  float o[HPW][NCH][8];
+  float m[HPW], l[HPW];
+#pragma unroll
+  for (int hh = 0; hh < HPW; ++hh) {
+    m[hh] = -INFINITY;
+    l[hh] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[hh][i][e] = 0.f;
+  }
+  const float log2e_cap = la.softcap > 0.f ? 1.4426950408889634f : 0.f;
+
+  for (int j = start + kg; j < end; j += KW) {
+    const size_t rowoff = ((static_cast<size_t>(b) * da.max_len + j) * la.Hkv + kvh) * D;
+    float kr[NCH][8];
+    load_row<NCH>(da.k + rowoff, lane, kr);
+    float kx[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kx[i][e] = kr[i][e];
+    transform_row<NCH>(kx, lane, j, la, la.k_norm_w, da.status);
+    float s[HPW];
+#pragma unroll
+    for (int hh = 0; hh < HPW; ++hh) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = fmaf(qreg[hh][i][e], kx[i][e], acc);
+      s[hh] = warp_sum(acc);
+      if (la.softcap > 0.f) {
+        // logits are in log2 units here: cap the natural-unit value c*tanh(x/c)
+        const float nat = s[hh] / 1.4426950408889634f;
+        s[hh] = la.softcap * tanhf(nat / la.softcap) * log2e_cap;
+      }
+    }
+    if (!la.k_eq_v) load_row<NCH>(da.v + rowoff, lane, kr);
+#pragma unroll
+    for (int hh = 0; hh < HPW; ++hh) {
+      const float mn = fmaxf(m[hh], s[hh]);
+      const float alpha = ex2(m[hh] - mn);
+      const float p = ex2(s[hh] - mn);
+      l[hh] = l[hh] * alpha + p;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[hh][i][e] = fmaf(o[hh][i][e], alpha, p * kr[i][e]);
+      m[hh] = mn;
+    }
+  }
+
+#pragma unroll
+  for (int hh = 0; hh < HPW; ++hh) {
+    if (lane == 0) {
+      pm[warp * HPW + hh] = m[hh];
+      pl[warp * HPW + hh] = l[hh];
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) po[(warp * HPW + hh) * D + 8 * (lane + 32 * i) + e] = o[hh][i][e];
+  }
+  __syncthreads();
+
+  // merge the KW key lanes of each head, write this CTA's partial
+  for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+    const int h = idx / D, d = idx % D;
+    const int g = h / HPW, hh = h % HPW;
+    float M = -INFINITY;
+    for (int k2 = 0; k2 < KW; ++k2) M = fmaxf(M, pm[(k2 * NHG + g) * HPW + hh]);
+    float num = 0.f, den = 0.f;
+    for (int k2 = 0; k2 < KW; ++k2) {
+      const int wi = (k2 * NHG + g) * HPW + hh;
+      const float lw = pl[wi];
+      if (lw > 0.f) {
+        const float f = ex2(pm[wi] - M);
+        num += f * po[wi * D + d];
+        den += f * lw;
+      }
+    }
+    const size_t slot = (head0 + h) * da.nsplit + split;
+    da.part_o[slot * D + d] = num;
+    if (d == 0) {
+      da.part_ml[slot * 2] = M;
+      da.part_ml[slot * 2 + 1] = den;
+    }
+  }
+}
+
+// Merge the per-chunk partials of one (b, h) row.
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs da, LayerArgs la) {
+  constexpr int PER = D / 128;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const size_t base = (static_cast<size_t>(b) * la.H + h) * da.nsplit;
+  float M = -INFINITY;
+  for (int s = 0; s < da.nsplit; ++s) {
+    const float l = da.part_ml[(base + s) * 2 + 1];
+    if (l > 0.f) M = fmaxf(M, da.part_ml[(base + s) * 2]);
+  }
+  float num[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) num[e] = 0.f;
+  float den = 0.f;
+  for (int s = 0; s < da.nsplit; ++s) {
+    const float l = da.part_ml[(base + s) * 2 + 1];
+    if (!(l > 0.f)) continue;
+    const float f = ex2(da.part_ml[(base + s) * 2] - M);
+    den += f * l;
+    const float* src = da.part_o + (base + s) * D + threadIdx.x * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) num[e] += f * src[e];
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  bf16* dst = da.out + (static_cast<size_t>(b) * la.H + h) * D + threadIdx.x * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2) {
+    *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(num[e] * inv, num[e + 1] * inv);
+  }
+}
+
+void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk) {
+  (void)B;
+  const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
+  const int c = la.window > 0 ? 256 : 1024;
+  *chunk = c;
+  *nsplit = (span + c - 1) / c;
+}
+
+template <int NCH, int HPW>
+static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  constexpr int D = NCH * 256;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(la.G) * D + 2 * kDecodeWarps * HPW +
+                                       static_cast<size_t>(kDecodeWarps) * HPW * D);
+  auto kern = decode_split_kernel<NCH, HPW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(da.nsplit, la.Hkv, da.B);
+  kern<<<grid, kDecodeWarps * 32, smem, s>>>(da, la);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  const int hpw = la.G <= 2 ? la.G : la.G / 4;
+  if (la.D == 256) {
+    switch (hpw) {
+      case 1: return run_decode_split<1, 1>(da, la, s);
+      case 2: return run_decode_split<1, 2>(da, la, s);
+      case 4: return run_decode_split<1, 4>(da, la, s);
+    }
+  } else {
+    switch (hpw) {
+      case 1: return run_decode_split<2, 1>(da, la, s);
+      case 2: return run_decode_split<2, 2>(da, la, s);
+      case 4: return run_decode_split<2, 4>(da, la, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  if (la.D == 256)
+    decode_combine_kernel<256><<<dim3(la.H, da.B), 128, 0, s>>>(da, la);
+  else
+    decode_combine_kernel<512><<<dim3(la.H, da.B), 128, 0, s>>>(da, la);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded wait: nothing ever arrives on the barrier.
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(uint32_t* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, timeout_ns, status, &abort_flag);
+  __syncthreads();
+}
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace gattn

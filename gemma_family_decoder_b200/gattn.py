@@ -1,0 +1,254 @@
+"""Thin ctypes binding of libgattn (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers and the current
+CUDA stream to the C ABI declared in ``include/gattn.h``; all arithmetic runs
+in the library's CUDA kernels.  There is no fallback: if ``libgattn.so`` is
+missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgattn.so")
+
+GATTN_OK = 0
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
+                5: "TIMEOUT", 6: "DEVICE_BOUNDS"}
+
+NORM_NONE, NORM_ONE_PLUS_W, NORM_W = 0, 1, 2
+
+EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_rope_table_bytes",
+           "gattn_rope_table_fill", "gattn_workspace_init", "gattn_prefill_workspace_size",
+           "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
+           "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events")
+
+
+class GattnError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({msg})")
+        self.status = status
+
+
+class GattnCfg(ctypes.Structure):
+    """Mirror of ``gattn_cfg`` (include/gattn.h)."""
+    _fields_ = [
+        ("num_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
+        ("rotary_fraction", ctypes.c_float),
+        ("rope_freq_dim", ctypes.c_int32),
+        ("rope_table", ctypes.c_void_p),
+        ("rope_max_pos", ctypes.c_int32),
+        ("softcap", ctypes.c_float),
+        ("scalar", ctypes.c_float),
+        ("k_eq_v", ctypes.c_int32),
+        ("qk_norm", ctypes.c_int32),
+        ("norm_eps", ctypes.c_float),
+        ("q_norm_w", ctypes.c_void_p),
+        ("k_norm_w", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgattn.so (built by ``python -m gemma_family_decoder_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libgattn.so not found at {LIB_PATH}; build it with "
+                              "`python -m gemma_family_decoder_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_float
+        L.gattn_version.restype = ctypes.c_char_p
+        L.gattn_status_string.restype = ctypes.c_char_p
+        L.gattn_status_string.argtypes = [ctypes.c_int]
+        L.gattn_last_error.restype = ctypes.c_char_p
+        L.gattn_rope_table_bytes.restype = sz
+        L.gattn_rope_table_bytes.argtypes = [i32, i32]
+        L.gattn_rope_table_fill.restype = ctypes.c_int
+        L.gattn_rope_table_fill.argtypes = [vp, f32, i32, i32, i32, vp]
+        L.gattn_workspace_init.restype = ctypes.c_int
+        L.gattn_workspace_init.argtypes = [vp, sz, vp]
+        L.gattn_prefill_workspace_size.restype = sz
+        L.gattn_prefill_workspace_size.argtypes = [ctypes.POINTER(GattnCfg), i32, i32]
+        L.gattn_prefill.restype = ctypes.c_int
+        L.gattn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz, vp]
+        L.gattn_decode_workspace_size.restype = sz
+        L.gattn_decode_workspace_size.argtypes = [ctypes.POINTER(GattnCfg), i32, i32]
+        L.gattn_decode.restype = ctypes.c_int
+        L.gattn_decode.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz, vp]
+        L.gattn_check.restype = ctypes.c_int
+        L.gattn_check.argtypes = [vp, vp]
+        L.gattn_selftest_wait_timeout.restype = ctypes.c_int
+        L.gattn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
+        L.gattn_set_wait_timeout_us.restype = None
+        L.gattn_set_wait_timeout_us.argtypes = [ctypes.c_uint32]
+        L.gattn_set_profile_events.restype = None
+        L.gattn_set_profile_events.argtypes = [vp, vp]
+        _lib = L
+    return _lib
+
+
+def _raise_if(status: int, where: str):
+    if status != GATTN_OK:
+        raise GattnError(status, where, lib().gattn_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if t.dtype != dtype or t.dim() != ndim or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of rank {ndim}, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+@dataclass
+class LayerSpec:
+    """Host description of one attention layer (the fields of ``gattn_cfg``)."""
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    window: int = 0
+    rope_theta: float = 10000.0
+    rotary_fraction: float = 1.0
+    rope_freq_dim: int = 0
+    softcap: float = 0.0
+    scalar: float = 256.0
+    k_eq_v: bool = False
+    qk_norm: int = NORM_NONE
+    norm_eps: float = 1e-6
+
+    @property
+    def rot_dim(self) -> int:
+        return int(round(self.rotary_fraction * self.head_dim))
+
+    @classmethod
+    def of(cls, obj) -> "LayerSpec":
+        return cls(**{f: getattr(obj, f) for f in cls.__dataclass_fields__})
+
+
+def rope_table(theta: float, rot_dim: int, freq_dim: int, max_pos: int, device="cuda",
+               stream=None) -> torch.Tensor:
+    """Device (cos, sin) table [max_pos][rot_dim/2][2] fp32 built by the library."""
+    n = lib().gattn_rope_table_bytes(max_pos, rot_dim)
+    if n == 0:
+        raise ValueError("invalid rope table size")
+    tab = torch.empty(n // 4, dtype=torch.float32, device=device)
+    _raise_if(lib().gattn_rope_table_fill(_ptr(tab), theta, rot_dim, freq_dim, max_pos,
+                                          _stream(stream)), "gattn_rope_table_fill")
+    return tab
+
+
+class AttentionLayer:
+    """A layer's device-side constants (RoPE table, QK-norm gains) and its cfg."""
+
+    def __init__(self, spec: LayerSpec, max_pos: int, w_q: Optional[torch.Tensor] = None,
+                 w_k: Optional[torch.Tensor] = None, device="cuda"):
+        self.spec = spec
+        self.max_pos = max_pos
+        R = spec.rot_dim
+        F = spec.rope_freq_dim or spec.head_dim
+        self.table = rope_table(spec.rope_theta, R, F, max_pos, device) if R > 0 else None
+        self.w_q = None if w_q is None else w_q.to(device=device, dtype=torch.float32).contiguous()
+        self.w_k = None if w_k is None else w_k.to(device=device, dtype=torch.float32).contiguous()
+        self.cfg = GattnCfg(
+            num_heads=spec.num_heads, num_kv_heads=spec.num_kv_heads, head_dim=spec.head_dim,
+            window=spec.window, rope_theta=spec.rope_theta, rotary_fraction=spec.rotary_fraction,
+            rope_freq_dim=spec.rope_freq_dim,
+            rope_table=None if self.table is None else self.table.data_ptr(),
+            rope_max_pos=max_pos if R > 0 else 0, softcap=spec.softcap, scalar=spec.scalar,
+            k_eq_v=int(spec.k_eq_v), qk_norm=spec.qk_norm, norm_eps=spec.norm_eps,
+            q_norm_w=None if self.w_q is None else self.w_q.data_ptr(),
+            k_norm_w=None if self.w_k is None else self.w_k.data_ptr())
+
+    # -- workspaces --------------------------------------------------------------
+    def prefill_workspace(self, batch: int, seq_len: int, device="cuda") -> torch.Tensor:
+        n = lib().gattn_prefill_workspace_size(ctypes.byref(self.cfg), batch, seq_len)
+        if n == 0:
+            raise GattnError(1, "gattn_prefill_workspace_size", "invalid cfg or sizes")
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+        _raise_if(lib().gattn_workspace_init(_ptr(ws), n, _stream()), "gattn_workspace_init")
+        return ws
+
+    def decode_workspace(self, batch: int, max_len: int, device="cuda") -> torch.Tensor:
+        n = lib().gattn_decode_workspace_size(ctypes.byref(self.cfg), batch, max_len)
+        if n == 0:
+            raise GattnError(1, "gattn_decode_workspace_size", "invalid cfg or sizes")
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+        _raise_if(lib().gattn_workspace_init(_ptr(ws), n, _stream()), "gattn_workspace_init")
+        return ws
+
+    # -- the two entry points ---------------------------------------------------
+    def prefill(self, q, k, v=None, positions=None, out=None, workspace=None, stream=None):
+        """gattn_prefill: q [B,S,H,D], k/v [B,S,Hkv,D] bf16, positions [B,S] int32."""
+        _need(q, "q", torch.bfloat16, 4)
+        _need(k, "k", torch.bfloat16, 4)
+        if v is not None:
+            _need(v, "v", torch.bfloat16, 4)
+        B, S = q.shape[0], q.shape[1]
+        if positions is None and self.spec.rot_dim > 0:
+            raise ValueError("positions are required when RoPE is on")
+        if positions is not None:
+            _need(positions, "positions", torch.int32, 2)
+        out = torch.empty_like(q) if out is None else out
+        ws = self.prefill_workspace(B, S, q.device) if workspace is None else workspace
+        _raise_if(lib().gattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(out), B, S,
+                                      ctypes.byref(self.cfg), _ptr(ws), ws.numel(), _stream(stream)),
+                  "gattn_prefill")
+        return out
+
+    def decode(self, q, k_cache, v_cache=None, seq_lens=None, out=None, workspace=None, stream=None):
+        """gattn_decode: q [B,H,D], caches [B,Lmax,Hkv,D] bf16 (raw keys/values), seq_lens [B] int32."""
+        _need(q, "q", torch.bfloat16, 3)
+        _need(k_cache, "k_cache", torch.bfloat16, 4)
+        if v_cache is not None:
+            _need(v_cache, "v_cache", torch.bfloat16, 4)
+        _need(seq_lens, "seq_lens", torch.int32, 1)
+        B, Lmax = k_cache.shape[0], k_cache.shape[1]
+        out = torch.empty_like(q) if out is None else out
+        ws = self.decode_workspace(B, Lmax, q.device) if workspace is None else workspace
+        _raise_if(lib().gattn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(out),
+                                     B, Lmax, ctypes.byref(self.cfg), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "gattn_decode")
+        return out
+
+
+def check(workspace: torch.Tensor, stream=None) -> int:
+    """gattn_check: synchronise, read and clear the status word; returns the status code."""
+    return lib().gattn_check(_stream(stream), _ptr(workspace))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, timeout_us: int, stream=None):
+    _raise_if(lib().gattn_selftest_wait_timeout(_ptr(workspace), workspace.numel(), timeout_us,
+                                                _stream(stream)), "gattn_selftest_wait_timeout")
+
+
+def set_wait_timeout_us(us: int):
+    lib().gattn_set_wait_timeout_us(us)
+
+
+def set_profile_events(start=None, stop=None):
+    """Time the main kernel of later calls: ``start``/``stop`` are torch.cuda.Event (or None)."""
+    lib().gattn_set_profile_events(None if start is None else ctypes.c_void_p(start.cuda_event),
+                                   None if stop is None else ctypes.c_void_p(stop.cuda_event))
+
+
+def version() -> str:
+    return lib().gattn_version().decode()

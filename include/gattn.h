@@ -1,0 +1,182 @@
+/*
+ * libgattn -- Gemma 1-4 decoder self-attention forward on one NVIDIA B200 (sm_100a).
+ *
+ * The layer computed by both entry points, step by step:
+ *   1. QK-norm: x / sqrt(mean(x^2) + eps) * g per head over head_dim, with
+ *      g = 1 + w (Gemma 3's usual gain) or g = w (KerasFormers "Gemma 4",
+ *      What changed: plain-weight RMSNorm).  QK-norm itself: Atlas "Gemma 4"
+ *      summary (RMSNorm pre/post-norm + QK-norm).
+ *   2. Rotary embedding on the first R = rotary_fraction * head_dim dims,
+ *      rotate-half pairs (t, t + R/2), angle pos * theta^(-2t/F); dims past R
+ *      pass through unchanged (KerasFormers "Gemma 4", What changed: zero-pad
+ *      partial rope; KerasFormers "Gemma 3", What changed: dual RoPE bases).
+ *   3. Logits s = (q~ . k~) * scalar^(-1/2) (ZeroModels "Gemma 2", API table:
+ *      query_pre_attn_scalar).
+ *   4. Optional cap s = c * tanh(s / c) (ZeroModels "Gemma 2", logit
+ *      softcapping bullet).
+ *   5. Causal mask, optionally a sliding window: key j is visible to query i
+ *      iff j <= i and (window == 0 or i - j < window) on token indices
+ *      (ZeroModels "Gemma 2", alternating attention bullet).
+ *   6. Softmax over visible keys, weighted sum of values.  With k_eq_v the
+ *      values are the raw key tensor (KerasFormers "Gemma 4", What changed:
+ *      K=V global MQA with tied key and value projections).
+ *   7. Query head h reads key/value head h / (num_heads / num_kv_heads)
+ *      (GQA; MQA when num_kv_heads == 1: KerasFormers "Gemma", API table).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no state besides a per-device
+ *     cache of attributes.  Pointers must be 16-byte aligned.
+ *   - bf16 tensors are passed as gattn_bf16 (raw IEEE bfloat16 bits).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; host arguments (cfg) are read during
+ *     the call only.
+ *   - Arguments are validated on the host before any launch; a failing check
+ *     returns a gattn_status code and enqueues nothing.  Nothing aborts.
+ *   - Errors found by the kernels themselves (a position outside the RoPE
+ *     table, a sequence length outside [1, max_len], a bounded wait that ran
+ *     out) are recorded in a status word at the start of the workspace and
+ *     are read (and cleared) by gattn_check.
+ */
+#ifndef GATTN_H_
+#define GATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t gattn_bf16;        /* raw bfloat16 storage */
+typedef struct CUstream_st* gattn_stream; /* same type as cudaStream_t */
+
+typedef enum {
+  GATTN_OK = 0,
+  GATTN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or cfg field */
+  GATTN_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. head_dim not 256/512) */
+  GATTN_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  GATTN_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  GATTN_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out (device) */
+  GATTN_ERR_DEVICE_BOUNDS = 6  /* a kernel saw an out-of-range index (device) */
+} gattn_status;
+
+typedef enum {
+  GATTN_NORM_NONE = 0,
+  GATTN_NORM_ONE_PLUS_W = 1,   /* gain 1 + w */
+  GATTN_NORM_W = 2             /* gain w */
+} gattn_norm;
+
+/* Layer description.  Read during the call only. */
+typedef struct {
+  int32_t num_heads;        /* H query heads                                    */
+  int32_t num_kv_heads;     /* Hkv key/value heads; H % Hkv == 0                */
+  int32_t head_dim;         /* D; 256 or 512                                    */
+  int32_t window;           /* 0 = full causal; else keys with i - j < window   */
+  float rope_theta;         /* RoPE base (1e4 local, 1e6 global)                */
+  float rotary_fraction;    /* R = fraction * D rotated dims; 0 = no RoPE.
+                               R must be a multiple of 16                       */
+  int32_t rope_freq_dim;    /* F in theta^(-2t/F); 0 means head_dim             */
+  const float* rope_table;  /* device table from gattn_rope_table_fill for the
+                               same (theta, R, F); NULL iff R == 0              */
+  int32_t rope_max_pos;     /* rows in rope_table; positions must be below it   */
+  float softcap;            /* c > 0 caps logits at c * tanh(s / c); 0 = off    */
+  float scalar;             /* query_pre_attn_scalar; scale = scalar^(-1/2) > 0 */
+  int32_t k_eq_v;           /* 1: values are the key tensor (v pointer NULL or
+                               equal to k)                                      */
+  int32_t qk_norm;          /* gattn_norm                                       */
+  float norm_eps;           /* RMSNorm epsilon (1e-6 in every Gemma card)       */
+  const float* q_norm_w;    /* device fp32 [D], shared by heads; NULL iff NONE  */
+  const float* k_norm_w;    /* device fp32 [D]; NULL iff NONE                   */
+} gattn_cfg;
+
+/* ---- RoPE table ---------------------------------------------------------
+ * Table of (cos, sin) pairs, fp32, layout [max_pos][rot_dim/2][2], with
+ * angle(p, t) = p * theta^(-2t/freq_dim) evaluated in double precision and
+ * rounded once to fp32.  Build it once per (theta, rot_dim, freq_dim) and
+ * pass it in gattn_cfg.rope_table.
+ * gattn_rope_table_bytes returns 0 for invalid sizes.
+ * gattn_rope_table_fill returns INVALID_ARG for a NULL/misaligned table,
+ * theta <= 0, rot_dim odd or <= 0, freq_dim <= 0 or max_pos <= 0. */
+size_t gattn_rope_table_bytes(int32_t max_pos, int32_t rot_dim);
+int gattn_rope_table_fill(float* table, float theta, int32_t rot_dim, int32_t freq_dim,
+                          int32_t max_pos, gattn_stream stream);
+
+/* ---- workspace -----------------------------------------------------------
+ * Every compute call takes a caller-owned device workspace.  Its first 256
+ * bytes hold the status word; gattn_workspace_init zeroes them (call it once
+ * after allocating).  Calls that share a workspace must be ordered on one
+ * stream. */
+int gattn_workspace_init(void* workspace, size_t ws_bytes, gattn_stream stream);
+
+/* ---- prefill --------------------------------------------------------------
+ * Self-attention of a whole prompt.
+ *   q         [batch][seq_len][H][D]    bf16, row-major ("BSHD")
+ *   k         [batch][seq_len][Hkv][D]  bf16
+ *   v_or_null [batch][seq_len][Hkv][D]  bf16; NULL (or == k) when cfg->k_eq_v
+ *   positions [batch][seq_len]          int32 RoPE positions, in [0, rope_max_pos)
+ *                                       (may be NULL when R == 0)
+ *   out       [batch][seq_len][H][D]    bf16, written completely
+ * The mask works on token indices 0..seq_len-1; positions drive RoPE only.
+ * workspace: at least gattn_prefill_workspace_size(cfg, batch, seq_len) bytes.
+ * Returns GATTN_OK once the kernels are enqueued. */
+size_t gattn_prefill_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t seq_len);
+int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
+                  const int32_t* positions, gattn_bf16* out, int32_t batch, int32_t seq_len,
+                  const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream);
+
+/* ---- decode ----------------------------------------------------------------
+ * One decode step: query b (at position seq_lens[b]-1) against cache rows
+ * [0, seq_lens[b]) of its own cache.  Caches hold RAW keys/values (before
+ * QK-norm and RoPE); cached key j sits at position j.
+ *   q               [batch][H][D]            bf16
+ *   k_cache         [batch][max_len][Hkv][D] bf16
+ *   v_cache_or_null [batch][max_len][Hkv][D] bf16; NULL (or == k_cache) when k_eq_v
+ *   seq_lens        [batch] int32 in [1, max_len] (device); rows outside it write zeros
+ *                   and flag GATTN_ERR_DEVICE_BOUNDS
+ *   out             [batch][H][D]            bf16
+ * Only the visible rows (the last `window` rows when windowed) are read.
+ * workspace: at least gattn_decode_workspace_size(cfg, batch, max_len) bytes. */
+size_t gattn_decode_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t max_len);
+int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf16* v_cache_or_null,
+                 const int32_t* seq_lens, gattn_bf16* out, int32_t batch, int32_t max_len,
+                 const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream);
+
+/* ---- status --------------------------------------------------------------------
+ * gattn_check synchronises `stream`, reads and clears the workspace status
+ * word, and returns GATTN_ERR_TIMEOUT or GATTN_ERR_DEVICE_BOUNDS if a kernel
+ * recorded one since the last check (timeout wins), else GATTN_OK (or
+ * GATTN_ERR_CUDA if synchronising failed). */
+int gattn_check(gattn_stream stream, void* workspace);
+const char* gattn_status_string(int status);
+/* Message for the last failing call on this host thread ("" if none). */
+const char* gattn_last_error(void);
+
+/* ---- self-test hooks ----------------------------------------------------------
+ * gattn_selftest_wait_timeout launches one CTA that waits, with the library's
+ * bounded-wait helper and a limit of `timeout_us` microseconds, on an
+ * mbarrier that nothing ever arrives on; the wait runs out, the CTA records
+ * GATTN_ERR_TIMEOUT in the workspace status word and exits normally.  It lets
+ * a test check the timeout path without hanging or faulting a GPU.
+ * gattn_set_wait_timeout_us sets the limit every later kernel launch in this
+ * process uses for its mbarrier waits (default 2,000,000 us); 0 restores it. */
+int gattn_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint32_t timeout_us,
+                                gattn_stream stream);
+void gattn_set_wait_timeout_us(uint32_t timeout_us);
+
+/* ---- profiling hook ----------------------------------------------------------
+ * gattn_set_profile_events(start, stop): when both are non-NULL (cudaEvent_t
+ * handles), every later gattn_prefill / gattn_decode call on this host thread
+ * records `start` on its stream right before launching its main kernel (the
+ * tensor-core prefill kernel, or the decode split kernel) and `stop` right
+ * after it, so a caller can time that kernel alone with cudaEventElapsedTime.
+ * Passing NULLs turns it off.  The events stay owned by the caller. */
+void gattn_set_profile_events(void* start_event, void* stop_event);
+
+/* Library version string, e.g. "libgattn 0.1 sm_100a". */
+const char* gattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GATTN_H_ */

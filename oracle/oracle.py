@@ -182,13 +182,16 @@ def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None):
 
 # --- the layer: one decode step ----------------------------------------------
 
-def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, batches=None):
+def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, batches=None,
+                     first_rows=None):
     """One decode step (float64): query b at position L_b - 1 over cache rows [0, L_b).
 
     q [B,H,D]; k_cache / v_cache [B,Lmax,Hkv,D] raw (un-normed, un-rotated)
     keys and values, or a list of per-batch [L_b,Hkv,D] arrays; cached key j
     sits at position j.  ``batches`` restricts the output to those batch rows.
-    Returns [len(batches),H,D].
+    ``first_rows[b]`` (default 0) says the cache given for batch row b starts
+    at row first_rows[b]; the rows left out must all be masked, which is
+    asserted.  Returns [len(batches),H,D].
     """
     f = _layer_fields(cfg)
     q = _f64(q)
@@ -199,9 +202,11 @@ def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, bat
     out = np.zeros((len(batches), H, D))
     for n, b in enumerate(batches):
         L = int(seq_lens[b])
-        kc = _f64(k_cache[b])[:L]
-        vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:L]
-        pos_k = np.arange(L)
+        r0 = 0 if first_rows is None else int(first_rows[b])
+        assert r0 == 0 or not visible(L - 1, r0 - 1, f["W"]), "a visible cache row was left out"
+        kc = _f64(k_cache[b])[:L - r0]
+        vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:L - r0]
+        pos_k = np.arange(r0, L)
         kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],
                   f["rot"], f["theta"], f["F"])
         qt = rope(rms_norm(q[b], w_q, f["mode"], f["eps"]), np.array([L - 1]),

@@ -1,0 +1,122 @@
+"""The C ABI: the library loads, exports every function the header declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gemma_family_decoder_b200 as G
+from gemma_family_decoder_b200 import gattn
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gattn.h")
+ALIGNED = 0x10000  # a fake, 16-byte aligned device address: never dereferenced here
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gattn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_exports_agree():
+    L = G.lib()
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(gattn.EXPORTS)
+
+
+def test_cfg_struct_matches_header_layout():
+    # int32 x4, float x2, int32, (pad), ptr, int32, float x2, int32 x2, float, ptr x2
+    assert ctypes.sizeof(G.GattnCfg) == 80
+    assert G.GattnCfg.rope_table.offset == 32
+    assert G.GattnCfg.q_norm_w.offset == 64
+
+
+def cfg(**kw):
+    base = dict(num_heads=8, num_kv_heads=1, head_dim=256, window=0, rope_theta=1e4,
+                rotary_fraction=0.0, rope_freq_dim=0, rope_table=None, rope_max_pos=0,
+                softcap=0.0, scalar=256.0, k_eq_v=0, qk_norm=0, norm_eps=1e-6,
+                q_norm_w=None, k_norm_w=None)
+    base.update(kw)
+    return G.GattnCfg(**base)
+
+
+def prefill(c, q=ALIGNED, k=ALIGNED, v=ALIGNED, pos=ALIGNED, out=ALIGNED, B=1, S=16, ws=ALIGNED,
+            ws_bytes=1 << 30):
+    return G.lib().gattn_prefill(q, k, v, pos, out, B, S, ctypes.byref(c), ws, ws_bytes, None)
+
+
+def decode(c, q=ALIGNED, k=ALIGNED, v=ALIGNED, lens=ALIGNED, out=ALIGNED, B=1, Lmax=16, ws=ALIGNED,
+           ws_bytes=1 << 30):
+    return G.lib().gattn_decode(q, k, v, lens, out, B, Lmax, ctypes.byref(c), ws, ws_bytes, None)
+
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(head_dim=128), UNSUPPORTED),
+    (dict(num_heads=6, num_kv_heads=4), INVALID),
+    (dict(num_kv_heads=0), INVALID),
+    (dict(window=-1), INVALID),
+    (dict(rotary_fraction=0.25), INVALID),          # RoPE on without a table
+    (dict(rotary_fraction=0.3), INVALID),           # 76.8 dims
+    (dict(rotary_fraction=0.375), UNSUPPORTED),     # 96 dims: not a power of two
+    (dict(softcap=-1.0), INVALID),
+    (dict(scalar=0.0), INVALID),
+    (dict(qk_norm=3), INVALID),
+    (dict(qk_norm=1), INVALID),                     # weights missing
+    (dict(k_eq_v=2), INVALID),
+])
+def test_prefill_rejects_bad_cfg(over, code):
+    assert prefill(cfg(**over)) == code
+    assert G.lib().gattn_last_error()
+
+
+def test_prefill_rejects_bad_pointers_and_sizes():
+    c = cfg()
+    assert prefill(c, q=None) == INVALID
+    assert prefill(c, q=ALIGNED + 8) == INVALID
+    assert prefill(c, v=None) == INVALID
+    assert prefill(c, B=-1) == INVALID
+    assert prefill(c, ws=None) == WORKSPACE
+    assert prefill(c, ws_bytes=16) == WORKSPACE
+    ck = cfg(k_eq_v=1)
+    assert prefill(ck, v=ALIGNED + 4096) == INVALID  # tied keys/values but a different v
+    cr = cfg(rotary_fraction=1.0, rope_table=ALIGNED, rope_max_pos=64)
+    assert prefill(cr, pos=None) == INVALID
+
+
+def test_empty_problem_is_a_no_op():
+    assert prefill(cfg(), B=0) == 0
+    assert prefill(cfg(), S=0) == 0
+    assert decode(cfg(), B=0) == 0
+
+
+def test_decode_rejects_bad_args():
+    assert decode(cfg(num_heads=24, num_kv_heads=1)) == UNSUPPORTED   # group of 24
+    assert decode(cfg(), lens=None) == INVALID
+    assert decode(cfg(), Lmax=0) == INVALID
+    assert decode(cfg(), ws_bytes=8) == WORKSPACE
+
+
+def test_workspace_sizes():
+    L = G.lib()
+    c = cfg(rotary_fraction=1.0, rope_table=ALIGNED, rope_max_pos=2048)
+    n = L.gattn_prefill_workspace_size(ctypes.byref(c), 4, 2048)
+    assert n >= 4 * 2048 * 1 * 256 * 2            # transformed keys
+    assert L.gattn_prefill_workspace_size(ctypes.byref(cfg()), 4, 2048) >= 256
+    assert L.gattn_prefill_workspace_size(ctypes.byref(cfg(head_dim=100)), 4, 2048) == 0
+    assert L.gattn_decode_workspace_size(ctypes.byref(cfg()), 64, 32768) > 0
+    assert L.gattn_rope_table_bytes(32768, 128) == 32768 * 64 * 8
+    assert L.gattn_rope_table_bytes(16, 3) == 0
+
+
+def test_status_strings():
+    L = G.lib()
+    for code in range(7):
+        assert L.gattn_status_string(code)
+    assert G.version().startswith("libgattn")
