@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag)) {
+      const bool got = mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
@@ -276,19 +277,23 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         rs += p;
       }
       if (j >= 1) {
-        if (!mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag)) {
+        const bool got = mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (rescale) {
+        // tcgen05.ld/st are warp-collective: rescale when any row of the warp
+        // needs it, with factor 1 for the rows that do not
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < C::DV / 32; ++c) {
             uint32_t rr[32];
             tmem_ld32(tmem + lane_off + C::TM_O + c * 32, rr);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
             tmem_st32(tmem + lane_off + C::TM_O + c * 32, rr);
           }
           tmem_wait_st();
@@ -312,7 +317,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag)) {
+    const bool fin = ok && mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag);
+    if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* orow = P.out + ((static_cast<size_t>(b) * S + qi) * H + h) * D + dv_lo;
