@@ -278,6 +278,10 @@ def run_ours(args, world, rank, local):
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e in ev:  # torch creates the CUDA event at its first record; the library re-records it
+        e[2].record(stream)
+        e[3].record(stream)
+    torch.cuda.synchronize()
     sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     sampler.start()
     time.sleep(0.3)

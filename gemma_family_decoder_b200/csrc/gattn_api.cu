@@ -74,6 +74,8 @@ int resolve(const gattn_cfg* cfg, gattn::LayerArgs* la, bool need_ptrs) {
     if (!(cfg->norm_eps >= 0.f)) return fail(GATTN_ERR_INVALID_ARG, "norm_eps must be >= 0");
     if (need_ptrs && (!cfg->q_norm_w || !cfg->k_norm_w))
       return fail(GATTN_ERR_INVALID_ARG, "QK-norm weights are NULL with qk_norm on");
+    if (need_ptrs && (!aligned16(cfg->q_norm_w) || !aligned16(cfg->k_norm_w)))
+      return fail(GATTN_ERR_INVALID_ARG, "QK-norm weights must be 16-byte aligned");
   }
   la->H = cfg->num_heads;
   la->Hkv = cfg->num_kv_heads;

@@ -2,12 +2,14 @@
 //
 // One CTA computes a 128-query tile of one head (and, for head_dim 512, one
 // 256-wide half of the value dims).  Warp roles:
-//   warps 0-3  query prologue (QK-norm + RoPE fused into the Q tile load), then
-//              per KV tile: S from TMEM -> scale, softcap, causal/window mask,
-//              online softmax with lazy rescale -> P (bf16) into shared memory;
-//              finally O / l -> bf16 -> global.
-//   warp 4     TMA producer: transformed-key tiles and value tiles into a
-//              two-stage shared-memory ring.
+//   warps 0-3  query prologue: the raw Q tile arrives by TMA and each thread
+//              applies QK-norm + RoPE to its own row in shared memory; then per
+//              KV tile: S from TMEM -> scale (and softcap) -> causal/window mask
+//              on boundary tiles only -> online softmax with lazy rescale ->
+//              P (bf16) into shared memory; finally O / l -> bf16 -> shared
+//              memory -> TMA store.
+//   warp 4     TMA producer: the Q tile, then transformed-key tiles and value
+//              tiles into a two-stage shared-memory ring.
 //   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM slot, then
 //              O += P V into the TMEM accumulator.
 // KV tiles entirely outside the causal window are never visited.
@@ -40,7 +42,7 @@ struct PrefillShape {
   static constexpr int OFF_RING = Q_BYTES;
   static constexpr int OFF_P = OFF_RING + NSTAGE * STAGE;
   static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int NBAR = 2 * NSTAGE + 8;
+  static constexpr int NBAR = 2 * NSTAGE + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr uint32_t TM_O = 0;
@@ -49,13 +51,14 @@ struct PrefillShape {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(TM_S1 + BN <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(Q_BYTES >= BM * DV * 2, "the output tile reuses the Q tile's shared memory");
 };
 
 struct PrefillKParams {
+  CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  const bf16* q;
-  bf16* out;
+  CUtensorMap tm_o;
   const int* positions;
   uint32_t* status;
   uint64_t timeout_ns;
@@ -63,7 +66,9 @@ struct PrefillKParams {
   LayerArgs la;
 };
 
-template <int D, int BN>
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, int BN, bool CAP>
 __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ PrefillKParams P) {
   using C = PrefillShape<D, BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -78,6 +83,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   uint64_t* o_done = p_full + 1;
   uint64_t* q_ready = o_done + 1;
   uint64_t* drain = q_ready + 1;
+  uint64_t* q_full = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -114,12 +120,15 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     mbar_init(o_done, 1);
     mbar_init(q_ready, 128);
     mbar_init(drain, 1);
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&P.tm_q);
     tma_prefetch_desc(&P.tm_k);
     tma_prefetch_desc(&P.tm_v);
+    tma_prefetch_desc(&P.tm_o);
   }
   if (warp == 5) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -137,39 +146,15 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     const int qi = q0 + t;
     const bool valid = qi < S;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    // query prologue: RMSNorm + RoPE in fp32, bf16 into the swizzled Q tile
-    {
-      uint8_t* qs = smem + C::OFF_Q;
-      const bf16* qrow = P.q + ((static_cast<size_t>(b) * S + qi) * H + h) * D;
-      int pos = 0;
-      float r = 1.f;
-      if (valid) {
-        if (la.rot > 0) {
-          pos = __ldg(P.positions + static_cast<size_t>(b) * S + qi);
-          if (pos < 0 || pos >= la.rope_max_pos) {
-            flag_status(P.status, kStatusBounds);
-            pos = pos < 0 ? 0 : la.rope_max_pos - 1;
-          }
-        }
-        if (la.qk_norm) {
-          float ss = 0.f;
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow) + c);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = unpack_bf16x2(w[e]);
-              ss += f.x * f.x + f.y * f.y;
-            }
-          }
-          r = rsqrtf(ss / static_cast<float>(D) + la.eps);
-        }
-      }
-      const float off = la.qk_norm == 1 ? 1.f : 0.f;
-      const int half = la.rot >> 1;
-      const float2* trow = la.rope_tab + static_cast<size_t>(pos) * (half > 0 ? half : 1);
-      auto load8 = [&](int c, float (&x)[8]) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(qrow) + c);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
+
+    // query prologue in place: RMSNorm + RoPE in fp32 on this thread's row
+    if (ok && valid && (la.rot > 0 || la.qk_norm)) {
+      uint8_t* qrow = smem + C::OFF_Q + t * 128;
+      auto chunk = [&](int c) -> uint4* {
+        return reinterpret_cast<uint4*>(qrow + (c >> 3) * C::SLAB128 + (((c & 7) ^ (t & 7)) << 4));
+      };
+      auto unpack8 = [](uint4 u, float (&x)[8]) {
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -177,89 +162,120 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           x[2 * e] = f.x;
           x[2 * e + 1] = f.y;
         }
-        if (la.qk_norm) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = x[e] * r * (__ldg(la.q_norm_w + 8 * c + e) + off);
-        }
       };
-      auto store8 = [&](int c, const float (&x)[8]) {
+      auto pack8 = [](const float (&x)[8]) {
         uint4 u;
         u.x = pack_bf16x2(x[0], x[1]);
         u.y = pack_bf16x2(x[2], x[3]);
         u.z = pack_bf16x2(x[4], x[5]);
         u.w = pack_bf16x2(x[6], x[7]);
-        const int phys = (c & 7) ^ (t & 7);
-        *reinterpret_cast<uint4*>(qs + (c >> 3) * C::SLAB128 + t * 128 + phys * 16) = u;
+        return u;
       };
-      for (int c = 0; c < D / 8; ++c) {
-        float x[8];
-        if (!valid) {
+      float r = 1.f;
+      if (la.qk_norm) {
+        float ss = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          float x[8];
+          unpack8(*chunk(c), x);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = 0.f;
-          store8(c, x);
-        } else if (8 * c < la.rot) {
-          if (8 * c >= half) continue;  // written with its partner
-          const int cp = c + (half >> 3);
-          float y[8];
-          load8(c, x);
-          load8(cp, y);
+          for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+        }
+        r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+      }
+      const float off = la.qk_norm == 1 ? 1.f : 0.f;
+      const float4* g4 = reinterpret_cast<const float4*>(la.q_norm_w);
+      auto gain8 = [&](int c, float (&x)[8]) {
+        if (!la.qk_norm) return;
+        const float4 g0 = __ldg(g4 + 2 * c), g1 = __ldg(g4 + 2 * c + 1);
+        x[0] *= r * (g0.x + off); x[1] *= r * (g0.y + off);
+        x[2] *= r * (g0.z + off); x[3] *= r * (g0.w + off);
+        x[4] *= r * (g1.x + off); x[5] *= r * (g1.y + off);
+        x[6] *= r * (g1.z + off); x[7] *= r * (g1.w + off);
+      };
+      const int h8 = la.rot >> 4;  // chunks in half the rotated slice
+      if (la.rot > 0) {
+        int pos = __ldg(P.positions + static_cast<size_t>(b) * S + qi);
+        if (pos < 0 || pos >= la.rope_max_pos) {
+          flag_status(P.status, kStatusBounds);
+          pos = pos < 0 ? 0 : la.rope_max_pos - 1;
+        }
+        const float4* trow = reinterpret_cast<const float4*>(la.rope_tab + static_cast<size_t>(pos) * (la.rot >> 1));
+#pragma unroll 2
+        for (int c = 0; c < h8; ++c) {
+          float x[8], y[8];
+          unpack8(*chunk(c), x);
+          unpack8(*chunk(c + h8), y);
+          gain8(c, x);
+          gain8(c + h8, y);
+          float cs[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 f = __ldg(trow + 4 * c + v);
+            cs[4 * v] = f.x; cs[4 * v + 1] = f.y; cs[4 * v + 2] = f.z; cs[4 * v + 3] = f.w;
+          }
           float xo[8], yo[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float2 cs = __ldg(trow + 8 * c + e);
-            xo[e] = x[e] * cs.x - y[e] * cs.y;
-            yo[e] = y[e] * cs.x + x[e] * cs.y;
+            const float co = cs[2 * e], si = cs[2 * e + 1];
+            xo[e] = x[e] * co - y[e] * si;
+            yo[e] = y[e] * co + x[e] * si;
           }
-          store8(c, xo);
-          store8(cp, yo);
-        } else {
-          load8(c, x);
-          store8(c, x);
+          *chunk(c) = pack8(xo);
+          *chunk(c + h8) = pack8(yo);
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(q_ready);
-    }
-
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const bool got = mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
+      if (la.qk_norm) {
+#pragma unroll 4
+        for (int c = 2 * h8; c < D / 8; ++c) {
+          float x[8];
+          unpack8(*chunk(c), x);
+          gain8(c, x);
+          *chunk(c) = pack8(x);
+        }
       }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+
+    // main loop over KV tiles
+    const float sl2 = la.scale_log2;
+    const float kcap = CAP ? la.scale / la.softcap : 0.f;
+    const float cap_l2 = CAP ? la.softcap * kLog2e : 0.f;
+    const int W = la.window;
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag));
+      if (!ok) break;
       tc_fence_after();
       const uint32_t scol = tmem + lane_off + ((j & 1) ? C::TM_S1 : C::TM_S0);
-      float s[BN];
+      uint32_t rr[BN / 32][32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(scol + c * 32, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
-      }
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_empty[j & 1]);
 
       const int key0 = k_first + j * BN;
-      float mx = -INFINITY;
+      const bool full_tile = (key0 + BN - 1 <= q0) && (q0 + C::BM <= S) &&
+                             (W <= 0 || (q0 + C::BM - 1) - key0 < W);
+      float x[BN];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        float x;
-        if (la.softcap > 0.f) {
-          x = la.softcap * tanhf(s[c] * la.scale / la.softcap) * 1.4426950408889634f;
-        } else {
-          x = s[c] * la.scale_log2;
-        }
-        const int key = key0 + c;
-        const bool vis = valid && key <= qi && (la.window <= 0 || qi - key < la.window);
-        x = vis ? x : -INFINITY;
-        s[c] = x;
-        mx = fmaxf(mx, x);
+      for (int i = 0; i < BN; ++i) {
+        const float s = __uint_as_float(rr[i >> 5][i & 31]);
+        x[i] = CAP ? cap_l2 * tanh_fast(s * kcap) : s;
       }
-      const float m_new = fmaxf(m, mx);
+      if (!full_tile) {
+        const int hi = valid ? qi - key0 : -1;            // visible iff i <= hi
+        const int lo = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
+#pragma unroll
+        for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, x[i]);
+      const float m_tile = CAP ? mx : mx * sl2;   // running max in log2 units
+      const float m_new = fmaxf(m, m_tile);
       float alpha = 1.f;
       bool rescale = false;
       float m_use = m;
@@ -270,18 +286,17 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       }
       const float mu = (m_use == -INFINITY) ? 0.f : m_use;
       float rs = 0.f;
+      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        const float p = ex2(s[c] - mu);
-        s[c] = p;
-        rs += p;
+      for (int i = 0; i < BN; i += 2) {
+        const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
+        const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
+        rs += p0 + p1;
+        pk[i >> 1] = pack_bf16x2(p0, p1);
       }
       if (j >= 1) {
-        const bool got = mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag));
+        if (!ok) break;
         tc_fence_after();
         // tcgen05.ld/st are warp-collective: rescale when any row of the warp
         // needs it, with factor 1 for the rows that do not
@@ -289,61 +304,68 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < C::DV / 32; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, rr);
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
-            tmem_st32(tmem + lane_off + C::TM_O + c * 32, rr);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
           }
           tmem_wait_st();
         }
       }
       l = (rescale ? l * alpha : l) + rs;
-      if (m_use != m) m = m_use;
+      m = m_use;
       // P row t (keys contiguous, 128-byte swizzle), 64 keys per slab
-      uint8_t* ps = smem + C::OFF_P;
+      uint8_t* ps = smem + C::OFF_P + t * 128;
 #pragma unroll
       for (int ch = 0; ch < BN / 8; ++ch) {
-        uint4 u;
-        u.x = pack_bf16x2(s[8 * ch + 0], s[8 * ch + 1]);
-        u.y = pack_bf16x2(s[8 * ch + 2], s[8 * ch + 3]);
-        u.z = pack_bf16x2(s[8 * ch + 4], s[8 * ch + 5]);
-        u.w = pack_bf16x2(s[8 * ch + 6], s[8 * ch + 7]);
-        const int phys = (ch & 7) ^ (t & 7);
-        *reinterpret_cast<uint4*>(ps + (ch >> 3) * C::SLAB128 + t * 128 + phys * 16) = u;
+        const uint4 u = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(ps + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (t & 7)) << 4)) = u;
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    const bool fin = ok && mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag);
-    if (__all_sync(0xffffffffu, fin)) {
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag));
+    if (ok) {
+      // epilogue: O / l -> bf16 into the (now idle) Q tile area, then TMA store
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* orow = P.out + ((static_cast<size_t>(b) * S + qi) * H + h) * D + dv_lo;
+      uint8_t* orow = smem + C::OFF_Q + t * 128;
 #pragma unroll 1
       for (int c = 0; c < C::DV / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, rr);
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
         tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
-            dst[v] = u;
-          }
+        for (int v = 0; v < 4; ++v) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+          u.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+          u.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+          u.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+          const int ch = 4 * c + v;
+          *reinterpret_cast<uint4*>(orow + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (t & 7)) << 4)) = u;
         }
+      }
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (t == 0) {
+#pragma unroll
+        for (int sl = 0; sl < C::DV / 64; ++sl)
+          tma_store_4d(&P.tm_o, smem + C::OFF_Q + sl * C::SLAB128, dv_lo + sl * 64, h, q0, b);
+        bulk_commit();
+        bulk_wait_read_all();
       }
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+      for (int sl = 0; sl < D / 64; ++sl)
+        tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
       int n = 0;
       auto load = [&](const CUtensorMap* tm, int d_base, int key0) -> bool {
         const int st = n % C::NSTAGE;
@@ -365,6 +387,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       }
       if (ok) load(&P.tm_v, dv_lo, k_first + (ntiles - 1) * BN);
       // let every issued copy land before the CTA can exit
+      mbar_wait(q_full, 0, tmo, P.status, nullptr);
       for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)
         mbar_wait(&full[i % C::NSTAGE], (i / C::NSTAGE) & 1, tmo, P.status, nullptr);
     }
@@ -435,14 +458,15 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   }
 }
 
-template <int D, int BN>
+template <int D, int BN, bool CAP>
 static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   using C = PrefillShape<D, BN>;
   PrefillKParams P;
-  if (!encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN)) return cudaErrorInvalidValue;
-  if (!encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN)) return cudaErrorInvalidValue;
-  P.q = pa.q;
-  P.out = pa.out;
+  if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, D, C::BM) ||
+      !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN) ||
+      !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN) ||
+      !encode_tmap_bshd(&P.tm_o, pa.out, pa.B, pa.S, la.H, D, C::BM))
+    return cudaErrorInvalidValue;
   P.positions = pa.positions;
   P.status = pa.status;
   P.timeout_ns = pa.timeout_ns;
@@ -451,7 +475,7 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.nqt = (pa.S + C::BM - 1) / C::BM;
   P.dv_splits = D / C::DV;
   P.la = la;
-  auto kern = prefill_kernel<D, BN>;
+  auto kern = prefill_kernel<D, BN, CAP>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -464,8 +488,9 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
 }
 
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
-  if (la.D == 256) return run_prefill<256, 128>(pa, la, s);
-  if (la.D == 512) return run_prefill<512, 64>(pa, la, s);
+  const bool cap = la.softcap > 0.f;
+  if (la.D == 256) return cap ? run_prefill<256, 128, true>(pa, la, s) : run_prefill<256, 128, false>(pa, la, s);
+  if (la.D == 512) return cap ? run_prefill<512, 64, true>(pa, la, s) : run_prefill<512, 64, false>(pa, la, s);
   return cudaErrorInvalidValue;
 }
 
