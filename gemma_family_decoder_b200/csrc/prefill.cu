@@ -6,12 +6,16 @@
 //              applies QK-norm + RoPE to its own row in shared memory; then per
 //              KV tile: S from TMEM -> scale (and softcap) -> causal/window mask
 //              on boundary tiles only -> online softmax with lazy rescale ->
-//              P (bf16) into shared memory; finally O / l -> bf16 -> shared
-//              memory -> TMA store.
+//              P (bf16) written back into the same TMEM columns; finally
+//              O / l -> bf16 -> shared memory -> TMA store.
 //   warp 4     TMA producer: the Q tile, then transformed-key tiles and value
 //              tiles into a two-stage shared-memory ring.
 //   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM slot, then
-//              O += P V into the TMEM accumulator.
+//              O += P V with P read from that slot, into the TMEM accumulator.
+// Because P lives in the S slot, the softmax of tile j+1 never waits for the
+// P V product of tile j (it waits only in the rare case that O must be
+// rescaled), and the tensor core runs Q K^T of tile j+1 while the softmax of
+// tile j is still being computed.
 // KV tiles entirely outside the causal window are never visited.
 //
 // Layer definition: KerasFormers "Gemma 4" (What changed: plain-weight RMSNorm,
@@ -37,11 +41,9 @@ struct PrefillShape {
   static constexpr int STAGE = 4 * SLAB_KV;      // 256 dims x BN rows
   static constexpr int SLAB128 = BM * 128;       // 64 dims x 128 rows
   static constexpr int Q_BYTES = (D / 64) * SLAB128;
-  static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = Q_BYTES;
-  static constexpr int OFF_P = OFF_RING + NSTAGE * STAGE;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * STAGE;
   static constexpr int NBAR = 2 * NSTAGE + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
@@ -78,9 +80,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   uint64_t* full = bars;
   uint64_t* empty = bars + C::NSTAGE;
   uint64_t* s_full = bars + 2 * C::NSTAGE;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_done = p_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
   uint64_t* q_ready = o_done + 1;
   uint64_t* drain = q_ready + 1;
   uint64_t* q_full = drain + 1;
@@ -114,9 +115,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
     }
-    mbar_init(p_full, 128);
     mbar_init(o_done, 1);
     mbar_init(q_ready, 128);
     mbar_init(drain, 1);
@@ -253,8 +253,6 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_empty[j & 1]);
 
       const int key0 = k_first + j * BN;
       const bool full_tile = (key0 + BN - 1 <= q0) && (q0 + C::BM <= S) &&
@@ -271,9 +269,13 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
         for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
       }
-      float mx = x[0];
+      float mxa[8];
 #pragma unroll
-      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, x[i]);
+      for (int a = 0; a < 8; ++a) mxa[a] = x[a];
+#pragma unroll
+      for (int i = 8; i < BN; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], x[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                             fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
       const float m_tile = CAP ? mx : mx * sl2;   // running max in log2 units
       const float m_new = fmaxf(m, m_tile);
       float alpha = 1.f;
@@ -285,47 +287,43 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         alpha = rescale ? ex2(m - m_new) : 0.f;
       }
       const float mu = (m_use == -INFINITY) ? 0.f : m_use;
-      float rs = 0.f;
-      uint32_t pk[BN / 2];
+      float rsa[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) rsa[a] = 0.f;
+      uint32_t pk[BN / 64][32];
 #pragma unroll
       for (int i = 0; i < BN; i += 2) {
         const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
         const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
-        rs += p0 + p1;
-        pk[i >> 1] = pack_bf16x2(p0, p1);
+        rsa[(i >> 1) & 7] += p0 + p1;
+        pk[i >> 6][(i >> 1) & 31] = pack_bf16x2(p0, p1);
       }
-      if (j >= 1) {
+      const float rs = ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+      // P (bf16 pairs) over the first BN/2 columns of this S slot
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c) tmem_st32(scol + c * 32, pk[c]);
+      // O must hold P V of every earlier tile before it is rescaled; that is
+      // the only case in which the softmax waits for the tensor core
+      if (__any_sync(0xffffffffu, rescale) && j >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        // tcgen05.ld/st are warp-collective: rescale when any row of the warp
-        // needs it, with factor 1 for the rows that do not
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float f = rescale ? alpha : 1.f;
+        const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < C::DV / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < C::DV / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
         }
       }
+      tmem_wait_st();
       l = (rescale ? l * alpha : l) + rs;
       m = m_use;
-      // P row t (keys contiguous, 128-byte swizzle), 64 keys per slab
-      uint8_t* ps = smem + C::OFF_P + t * 128;
-#pragma unroll
-      for (int ch = 0; ch < BN / 8; ++ch) {
-        const uint4 u = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(ps + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (t & 7)) << 4)) = u;
-      }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
     ok = ok && __all_sync(0xffffffffu, mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag));
     if (ok) {
@@ -421,26 +419,26 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         return true;
       };
       auto pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1, tmo, P.status, abort_flag)) return false;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, tmo, P.status, abort_flag)) return false;
         const int st = n % C::NSTAGE;
         if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sbase + C::OFF_RING + st * C::STAGE;
+        const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(
-              sbase + C::OFF_P + (kk >> 2) * C::SLAB128 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
-          mma_bf16_ss(tmem + C::TM_O, a, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[st]);
         ++n;
         mma_commit(o_done);
         return true;
       };
+      // issue order Q K^T(j), P V(j-1): the slot of tile j is rewritten by
+      // Q K^T(j+2) only after P V(j), which reads P from it, was issued
       for (int j = 0; j < ntiles && ok; ++j) {
-        if (j >= 2) ok = mbar_wait(&s_empty[j & 1], ((j >> 1) - 1) & 1, tmo, P.status, abort_flag);
-        if (ok) ok = qk(j);
+        ok = qk(j);
         if (ok && j >= 1) ok = pv(j - 1);
       }
       if (ok) pv(ntiles - 1);
