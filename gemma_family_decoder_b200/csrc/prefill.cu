@@ -9,7 +9,8 @@
 //              P (bf16) written back into the same TMEM columns; finally
 //              O / l -> bf16 -> shared memory -> TMA store.
 //   warp 4     TMA producer: the Q tile, then transformed-key tiles and value
-//              tiles into a two-stage shared-memory ring.
+//              tiles, one 64-dim box at a time, into a ring of box-sized slots
+//              (about one key tile plus one value tile of look-ahead).
 //   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM slot, then
 //              O += P V with P read from that slot, into the TMEM accumulator.
 // Because P lives in the S slot, the softmax of tile j+1 never waits for the
@@ -35,16 +36,17 @@ template <int D, int BN>
 struct PrefillShape {
   static constexpr int BM = 128;
   static constexpr int DV = 256;                 // value dims per CTA
-  static constexpr int NSTAGE = 2;
-  static constexpr int KSTAGES = D / 256;        // ring stages per key tile
-  static constexpr int SLAB_KV = BN * 128;       // one 64-dim TMA box of BN rows
-  static constexpr int STAGE = 4 * SLAB_KV;      // 256 dims x BN rows
+  static constexpr int SLAB_KV = BN * 128;       // one 64-dim TMA box of BN rows = one slot
+  static constexpr int KCH = D / 64;             // slots per key tile
+  static constexpr int VCH = DV / 64;            // slots per value tile
   static constexpr int SLAB128 = BM * 128;       // 64 dims x 128 rows
   static constexpr int Q_BYTES = (D / 64) * SLAB128;
+  static constexpr int NSTAGE = (227 * 1024 - Q_BYTES - 2048) / SLAB_KV;  // ring slots
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = Q_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + NSTAGE * STAGE;
+  static constexpr int OFF_BAR = OFF_RING + NSTAGE * SLAB_KV;
   static constexpr int NBAR = 2 * NSTAGE + 9;
+  static_assert(NSTAGE >= KCH + VCH, "ring must hold a key tile and a value tile");
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr uint32_t TM_O = 0;
@@ -365,25 +367,23 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       for (int sl = 0; sl < D / 64; ++sl)
         tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
       int n = 0;
-      auto load = [&](const CUtensorMap* tm, int d_base, int key0) -> bool {
+      auto load = [&](const CUtensorMap* tm, int d0, int key0) -> bool {
         const int st = n % C::NSTAGE;
         const uint32_t par = ((n / C::NSTAGE) & 1) ^ 1;
         if (!mbar_wait(&empty[st], par, tmo, P.status, abort_flag)) return false;
-        mbar_arrive_expect_tx(&full[st], C::STAGE);
-        uint8_t* dst = smem + C::OFF_RING + st * C::STAGE;
-#pragma unroll
-        for (int sub = 0; sub < 4; ++sub)
-          tma_load_4d(dst + sub * C::SLAB_KV, tm, &full[st], d_base + sub * 64, kvh, key0, b);
+        mbar_arrive_expect_tx(&full[st], C::SLAB_KV);
+        tma_load_4d(smem + C::OFF_RING + st * C::SLAB_KV, tm, &full[st], d0, kvh, key0, b);
         ++n;
         return true;
       };
+      // same order as the MMA issuer consumes them: K(j) then V(j-1)
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
         const int key0 = k_first + j * BN;
-        for (int ks = 0; ks < C::KSTAGES && ok; ++ks) ok = load(&P.tm_k, ks * 256, key0);
-        if (ok && j >= 1) ok = load(&P.tm_v, dv_lo, key0 - BN);
+        for (int c = 0; c < C::KCH && ok; ++c) ok = load(&P.tm_k, c * 64, key0);
+        for (int c = 0; c < C::VCH && ok && j >= 1; ++c) ok = load(&P.tm_v, dv_lo + c * 64, key0 - BN);
       }
-      if (ok) load(&P.tm_v, dv_lo, k_first + (ntiles - 1) * BN);
+      for (int c = 0; c < C::VCH && ok; ++c) ok = load(&P.tm_v, dv_lo + c * 64, k_first + (ntiles - 1) * BN);
       // let every issued copy land before the CTA can exit
       mbar_wait(q_full, 0, tmo, P.status, nullptr);
       for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)
@@ -393,24 +393,23 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
       int n = 0;
       bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
       tc_fence_after();
       auto qk = [&](int j) -> bool {
         const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
-        for (int ks = 0; ks < C::KSTAGES; ++ks) {
+        for (int c = 0; c < C::KCH; ++c) {
           const int st = n % C::NSTAGE;
           if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
           tc_fence_after();
-          const uint32_t kb = sbase + C::OFF_RING + st * C::STAGE;
+          const uint32_t kb = sbase + C::OFF_RING + st * C::SLAB_KV;
+          const uint32_t qb = sbase + C::OFF_Q + c * C::SLAB128;
 #pragma unroll
-          for (int kk = 0; kk < 16; ++kk) {
-            const int dim = ks * 256 + kk * 16;
-            const uint64_t a = smem_desc_sw128(
-                sbase + C::OFF_Q + (dim >> 6) * C::SLAB128 + (dim & 63) * 2, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * C::SLAB_KV + (kk & 3) * 32, 16, 1024);
-            mma_bf16_ss(s_tm, a, bd, idesc_qk, (ks | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t a = smem_desc_sw128(qb + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kb + kk * 32, 16, 1024);
+            mma_bf16_ss(s_tm, a, bd, idesc_qk, (c | kk) != 0);
           }
           mma_commit(&empty[st]);
           ++n;
@@ -420,18 +419,21 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       };
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, tmo, P.status, abort_flag)) return false;
-        const int st = n % C::NSTAGE;
-        if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vb = sbase + C::OFF_RING + st * C::STAGE;
         const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
+        for (int c = 0; c < C::VCH; ++c) {
+          const int st = n % C::NSTAGE;
+          if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t vb = sbase + C::OFF_RING + st * C::SLAB_KV;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
-          mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // 16 keys x 64 value dims, MN-major: key rows 128 B apart, 8-row groups 1 KB apart
+            const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 0, 1024);
+            mma_bf16_ts(tmem + C::TM_O + c * 64, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[st]);
+          ++n;
         }
-        mma_commit(&empty[st]);
-        ++n;
         mma_commit(o_done);
         return true;
       };
