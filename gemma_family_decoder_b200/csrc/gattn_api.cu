@@ -17,6 +17,8 @@ namespace {
 thread_local char g_last_error[512] = "";
 thread_local cudaEvent_t g_prof_start = nullptr;
 thread_local cudaEvent_t g_prof_stop = nullptr;
+thread_local void* g_trace_buf = nullptr;
+thread_local size_t g_trace_bytes = 0;
 uint64_t g_timeout_ns = 2000000ull * 1000ull;  // 2 s
 
 int fail(int code, const char* fmt, const char* detail = nullptr) {
@@ -249,6 +251,8 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   pa.S = seq_len;
   pa.status = status;
   pa.timeout_ns = gattn::wait_timeout_ns();
+  pa.trace = static_cast<unsigned long long*>(g_trace_buf);
+  pa.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
   cudaError_t e = gattn::launch_prefill(pa, la, s);
   if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
@@ -356,6 +360,11 @@ void gattn_set_profile_events(void* start_event, void* stop_event) {
     g_prof_start = nullptr;
     g_prof_stop = nullptr;
   }
+}
+
+void gattn_set_trace_buffer(void* device_buffer, size_t bytes) {
+  g_trace_buf = (device_buffer && bytes) ? device_buffer : nullptr;
+  g_trace_bytes = g_trace_buf ? bytes : 0;
 }
 
 int gattn_selftest_wait_timeout(void* workspace, size_t ws_bytes, uint32_t timeout_us,

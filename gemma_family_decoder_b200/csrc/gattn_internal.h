@@ -61,6 +61,8 @@ struct PrefillArgs {
   int B, S;
   uint32_t* status;
   uint64_t timeout_ns;
+  unsigned long long* trace;  // optional kernel timeline buffer (null = off)
+  size_t trace_bytes;
 };
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
 

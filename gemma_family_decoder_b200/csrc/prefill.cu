@@ -41,12 +41,14 @@ struct PrefillShape {
   static constexpr int VCH = DV / 64;            // slots per value tile
   static constexpr int SLAB128 = BM * 128;       // 64 dims x 128 rows
   static constexpr int Q_BYTES = (D / 64) * SLAB128;
-  static constexpr int NSTAGE = (227 * 1024 - Q_BYTES - 2048) / SLAB_KV;  // ring slots
+  // ring slots: a multiple of 4 so that every 4-slot value tile is contiguous
+  static constexpr int NSTAGE = ((227 * 1024 - Q_BYTES - 2048) / SLAB_KV) / 4 * 4;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * SLAB_KV;
-  static constexpr int NBAR = 2 * NSTAGE + 9;
+  static constexpr int NBAR = 2 * NSTAGE + 10;
   static_assert(NSTAGE >= KCH + VCH, "ring must hold a key tile and a value tile");
+  static_assert(KCH % 4 == 0 && VCH == 4 && NSTAGE % 4 == 0, "value tiles must not wrap the ring");
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr uint32_t TM_O = 0;
@@ -68,7 +70,16 @@ struct PrefillKParams {
   uint64_t timeout_ns;
   int B, S, nqt, dv_splits;
   LayerArgs la;
+  unsigned long long* trace;  // optional per-CTA event times (kTraceSlots each), or null
+  int trace_ctas;
 };
+
+// Optional timeline of one CTA (debug aid, off unless a trace buffer is set):
+// [0] start time (ns), [1] SM id, [2] KV tiles, [3] Q ready at the MMA warp,
+// [4] epilogue start, [5] end, [6] first key box landed, then per KV tile j
+// (j < 120): [8+j] S(j) seen by the softmax, [128+j] P(j) written,
+// [248+j] Q K^T(j) issued, [368+j] P V(j) issued; times relative to [0].
+constexpr int kTraceSlots = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -87,6 +98,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   uint64_t* q_ready = o_done + 1;
   uint64_t* drain = q_ready + 1;
   uint64_t* q_full = drain + 1;
+  uint64_t* o_final = q_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -123,6 +135,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     mbar_init(q_ready, 128);
     mbar_init(drain, 1);
     mbar_init(q_full, 1);
+    mbar_init(o_final, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -141,6 +154,19 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = P.timeout_ns;
+  unsigned long long* trace = (P.trace && static_cast<int>(blockIdx.x) < P.trace_ctas)
+                                  ? P.trace + static_cast<size_t>(blockIdx.x) * kTraceSlots : nullptr;
+  const uint64_t t_start = globaltimer_ns();
+  auto mark = [&](int slot) {
+    if (trace) trace[slot] = globaltimer_ns() - t_start;
+  };
+  if (trace && threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    trace[0] = t_start;
+    trace[1] = smid;
+    trace[2] = ntiles;
+  }
 
   if (warp < 4) {
     // ------------------------------------------------------------------ softmax
@@ -249,6 +275,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     for (int j = 0; j < ntiles && ok; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag));
       if (!ok) break;
+      if (t == 0 && j < 120) mark(8 + j);
       tc_fence_after();
       const uint32_t scol = tmem + lane_off + ((j & 1) ? C::TM_S1 : C::TM_S0);
       uint32_t rr[BN / 32][32];
@@ -305,7 +332,9 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(scol + c * 32, pk[c]);
       // O must hold P V of every earlier tile before it is rescaled; that is
-      // the only case in which the softmax waits for the tensor core
+      // the only case in which the softmax waits for the tensor core.  Seeing
+      // S(j) implies P V(j-2) is complete (it was issued before Q K^T(j)), so
+      // o_done is at most one phase behind and its parity wait is exact.
       if (__any_sync(0xffffffffu, rescale) && j >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag));
         if (!ok) break;
@@ -326,10 +355,12 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       m = m_use;
       tc_fence_before();
       mbar_arrive(&p_full[j & 1]);
+      if (t == 0 && j < 120) mark(128 + j);
     }
-    ok = ok && __all_sync(0xffffffffu, mbar_wait(o_done, (ntiles - 1) & 1, tmo, P.status, abort_flag));
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, tmo, P.status, abort_flag));
     if (ok) {
       // epilogue: O / l -> bf16 into the (now idle) Q tile area, then TMA store
+      if (t == 0) mark(4);
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint8_t* orow = smem + C::OFF_Q + t * 128;
@@ -393,15 +424,17 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
       int n = 0;
       bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
+      mark(3);
       tc_fence_after();
       auto qk = [&](int j) -> bool {
         const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
         for (int c = 0; c < C::KCH; ++c) {
           const int st = n % C::NSTAGE;
           if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
+          if (n == 0) mark(6);
           tc_fence_after();
           const uint32_t kb = sbase + C::OFF_RING + st * C::SLAB_KV;
           const uint32_t qb = sbase + C::OFF_Q + c * C::SLAB128;
@@ -415,26 +448,31 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           ++n;
         }
         mma_commit(&s_full[j & 1]);
+        if (j < 120) mark(248 + j);
         return true;
       };
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, tmo, P.status, abort_flag)) return false;
         const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
+        // the VCH value boxes sit in VCH consecutive slots (tiles are 4-slot aligned)
+        const int st0 = n % C::NSTAGE;
         for (int c = 0; c < C::VCH; ++c) {
-          const int st = n % C::NSTAGE;
-          if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t vb = sbase + C::OFF_RING + st * C::SLAB_KV;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            // 16 keys x 64 value dims, MN-major: key rows 128 B apart, 8-row groups 1 KB apart
-            const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 0, 1024);
-            mma_bf16_ts(tmem + C::TM_O + c * 64, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&empty[st]);
-          ++n;
+          const int st = st0 + c;
+          if (!mbar_wait(&full[st], ((n + c) / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
         }
+        tc_fence_after();
+        const uint32_t vb = sbase + C::OFF_RING + st0 * C::SLAB_KV;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // 16 keys x 256 value dims, MN-major: key rows 128 B apart, 8-row groups
+          // 1 KB apart, 64-dim boxes one slot apart
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
+          mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        for (int c = 0; c < C::VCH; ++c) mma_commit(&empty[st0 + c]);
+        n += C::VCH;
         mma_commit(o_done);
+        if (i < 120) mark(368 + i);
         return true;
       };
       // issue order Q K^T(j), P V(j-1): the slot of tile j is rewritten by
@@ -444,6 +482,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         if (ok && j >= 1) ok = pv(j - 1);
       }
       if (ok) pv(ntiles - 1);
+      mma_commit(o_final);
       // every MMA issued above has completed before TMEM is released
       mma_commit(drain);
       mbar_wait(drain, 0, tmo, P.status, nullptr);
@@ -456,6 +495,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) mark(5);
 }
 
 template <int D, int BN, bool CAP>
@@ -475,6 +515,8 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.nqt = (pa.S + C::BM - 1) / C::BM;
   P.dv_splits = D / C::DV;
   P.la = la;
+  P.trace = pa.trace;
+  P.trace_ctas = static_cast<int>(pa.trace_bytes / (kTraceSlots * sizeof(unsigned long long)));
   auto kern = prefill_kernel<D, BN, CAP>;
   static bool attr_set = false;
   if (!attr_set) {

@@ -26,7 +26,8 @@ NORM_NONE, NORM_ONE_PLUS_W, NORM_W = 0, 1, 2
 EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_rope_table_bytes",
            "gattn_rope_table_fill", "gattn_workspace_init", "gattn_prefill_workspace_size",
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
-           "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events")
+           "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
+           "gattn_set_trace_buffer")
 
 
 class GattnError(RuntimeError):
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.gattn_set_wait_timeout_us.argtypes = [ctypes.c_uint32]
         L.gattn_set_profile_events.restype = None
         L.gattn_set_profile_events.argtypes = [vp, vp]
+        L.gattn_set_trace_buffer.restype = None
+        L.gattn_set_trace_buffer.argtypes = [vp, sz]
         _lib = L
     return _lib
 
@@ -248,6 +251,14 @@ def set_profile_events(start=None, stop=None):
     """Time the main kernel of later calls: ``start``/``stop`` are torch.cuda.Event (or None)."""
     lib().gattn_set_profile_events(None if start is None else ctypes.c_void_p(start.cuda_event),
                                    None if stop is None else ctypes.c_void_p(stop.cuda_event))
+
+
+def set_trace_buffer(buf: Optional[torch.Tensor] = None):
+    """Record per-CTA prefill timelines into ``buf`` (int64 CUDA tensor), or stop (None)."""
+    if buf is None:
+        lib().gattn_set_trace_buffer(None, 0)
+    else:
+        lib().gattn_set_trace_buffer(ctypes.c_void_p(buf.data_ptr()), buf.numel() * buf.element_size())
 
 
 def version() -> str:

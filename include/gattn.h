@@ -173,6 +173,16 @@ void gattn_set_wait_timeout_us(uint32_t timeout_us);
  * Passing NULLs turns it off.  The events stay owned by the caller. */
 void gattn_set_profile_events(void* start_event, void* stop_event);
 
+/* gattn_set_trace_buffer(buf, bytes): when buf (a device buffer of `bytes`
+ * bytes, 8-byte aligned) is non-NULL, every later gattn_prefill call on this
+ * host thread has each of its first bytes/4096 CTAs write a timeline of 512
+ * 64-bit entries: [0] start time (ns, %globaltimer), [1] SM id, [2] key tiles,
+ * [3] Q ready, [4] epilogue start, [5] end, [6] first key box landed, and per
+ * key tile j < 120: [8+j] S(j) seen by the softmax, [128+j] P(j) written,
+ * [248+j] Q K^T(j) issued, [368+j] P V(j) issued, each in ns after [0].
+ * A debugging aid; NULL turns it off. */
+void gattn_set_trace_buffer(void* device_buffer, size_t bytes);
+
 /* Library version string, e.g. "libgattn 0.1 sm_100a". */
 const char* gattn_version(void);
 
