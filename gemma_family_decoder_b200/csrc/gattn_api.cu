@@ -123,6 +123,34 @@ namespace gattn {
 
 uint64_t wait_timeout_ns() { return g_timeout_ns; }
 
+int report_error(int code, const char* msg) { return fail(code, msg); }
+
+int check_decode_call(const gattn_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache_or_null, const int32_t* seq_lens, const void* out,
+                      int32_t batch, int32_t max_len, LayerArgs* la) {
+  g_last_error[0] = 0;
+  int st = resolve(cfg, la, true);
+  if (st != GATTN_OK) return st;
+  const int G = la->G;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+    return fail(GATTN_ERR_UNSUPPORTED, "decode supports num_heads / num_kv_heads in {1,2,4,8,16}");
+  if (batch < 0 || max_len <= 0) return fail(GATTN_ERR_INVALID_ARG, "batch must be >= 0 and max_len > 0");
+  if (!q || !k_cache || !out || !seq_lens)
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_cache, seq_lens and out must not be NULL");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out))
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_cache and out must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(seq_lens) & 3u)
+    return fail(GATTN_ERR_INVALID_ARG, "seq_lens must be 4-byte aligned");
+  if (la->k_eq_v) {
+    if (v_cache_or_null && v_cache_or_null != k_cache)
+      return fail(GATTN_ERR_INVALID_ARG, "k_eq_v: v_cache must be NULL or k_cache");
+  } else {
+    if (!v_cache_or_null) return fail(GATTN_ERR_INVALID_ARG, "v_cache is NULL without k_eq_v");
+    if (!aligned16(v_cache_or_null)) return fail(GATTN_ERR_INVALID_ARG, "v_cache must be 16-byte aligned");
+  }
+  return GATTN_OK;
+}
+
 bool encode_tmap_bshd(CUtensorMap* map, const void* base, int B, int S, int Hkv, int D,
                       int box_rows) {
   EncodeTiledFn fn = encode_fn();

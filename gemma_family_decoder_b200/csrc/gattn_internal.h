@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gattn.h"
+
 namespace gattn {
 
 // Fields shared by every kernel, resolved from gattn_cfg on the host.
@@ -68,6 +70,14 @@ cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStrea
 
 // Self-test: one CTA waits on an mbarrier nobody arrives on.
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t s);
+
+// Host checks of a decode call without its workspace arguments (the same
+// checks gattn_decode makes); fills `la`.  Returns a gattn_status.
+int check_decode_call(const gattn_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache_or_null, const int32_t* seq_lens, const void* out,
+                      int32_t batch, int32_t max_len, LayerArgs* la);
+// Record `msg` as this thread's last error and return `code`.
+int report_error(int code, const char* msg);
 
 // Wait limit used by every launch (ns).
 uint64_t wait_timeout_ns();

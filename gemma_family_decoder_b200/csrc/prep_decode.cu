@@ -9,6 +9,8 @@
 // second kernel merges them with the log-sum-exp rule.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "gattn_internal.h"
 #include "kernels/common.cuh"
 
@@ -424,4 +426,85 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStre
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Workspace-free decode.  Its split partials live in this file-scope device
+// array instead of a caller workspace; every GPU that loads the library keeps
+// the array until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  In host code the array's name is only a host-side handle.
+cudaError_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+}  // namespace
+
 }  // namespace gattn
+
+extern "C" int gattn_decode_noalloc(const gattn_bf16* q, const gattn_bf16* k_cache,
+                                    const gattn_bf16* v_cache_or_null, const int32_t* seq_lens,
+                                    gattn_bf16* out, int32_t batch, int32_t max_len,
+                                    const gattn_cfg* cfg, gattn_stream stream) {
+  using namespace gattn;
+  LayerArgs la;
+  int st = check_decode_call(cfg, q, k_cache, v_cache_or_null, seq_lens, out, batch, max_len, &la);
+  if (st != GATTN_OK) return st;
+  if (batch == 0) return GATTN_OK;
+
+  // the normal split plan, with fewer (longer) splits when its partials
+  // would not fit the scratch array
+  DecodeArgs da;
+  decode_plan(la, batch, max_len, &da.nsplit, &da.chunk);
+  const size_t per_split = static_cast<size_t>(batch) * la.H * (la.D + 2) * sizeof(float);
+  const size_t usable = kNoAllocScratchBytes - 512;  // room for two 256-byte roundings
+  const int max_split = static_cast<int>(usable / per_split);
+  if (max_split < 1)
+    return report_error(GATTN_ERR_UNSUPPORTED,
+                        "batch * num_heads * (head_dim + 2) * 4 bytes exceed the 16 MiB scratch "
+                        "of gattn_decode_noalloc; use gattn_decode with a workspace");
+  if (da.nsplit > max_split) {
+    const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
+    da.chunk = (span + max_split - 1) / max_split;
+    da.nsplit = (span + da.chunk - 1) / da.chunk;
+  }
+  void* base = nullptr;
+  cudaError_t e = noalloc_scratch_address(&base);
+  if (e != cudaSuccess) return report_error(GATTN_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch failed");
+  const size_t rows = static_cast<size_t>(batch) * la.H * da.nsplit;
+  da.part_o = static_cast<float*>(base);
+  da.part_ml = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + round256(rows * la.D * sizeof(float)));
+  da.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  da.k = reinterpret_cast<const __nv_bfloat16*>(k_cache);
+  da.v = la.k_eq_v ? da.k : reinterpret_cast<const __nv_bfloat16*>(v_cache_or_null);
+  da.seq_lens = seq_lens;
+  da.out = reinterpret_cast<__nv_bfloat16*>(out);
+  da.B = batch;
+  da.max_len = max_len;
+  da.status = nullptr;  // no status word: there is no workspace to hold one
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = launch_decode_split(da, la, s);
+  if (e == cudaSuccess) e = launch_decode_combine(da, la, s);
+  if (e != cudaSuccess) return report_error(GATTN_ERR_CUDA, cudaGetErrorString(e));
+  return GATTN_OK;
+}

@@ -27,7 +27,7 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_rope_table_fill", "gattn_workspace_init", "gattn_prefill_workspace_size",
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
-           "gattn_set_trace_buffer")
+           "gattn_set_trace_buffer", "gattn_decode_noalloc")
 
 
 class GattnError(RuntimeError):
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.gattn_set_profile_events.argtypes = [vp, vp]
         L.gattn_set_trace_buffer.restype = None
         L.gattn_set_trace_buffer.argtypes = [vp, sz]
+        L.gattn_decode_noalloc.restype = ctypes.c_int
+        L.gattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp]
         _lib = L
     return _lib
 
@@ -231,6 +233,22 @@ class AttentionLayer:
                                      B, Lmax, ctypes.byref(self.cfg), _ptr(ws), ws.numel(),
                                      _stream(stream)), "gattn_decode")
         return out
+
+
+def decode_noalloc(layer: "AttentionLayer", q, k_cache, v_cache=None, seq_lens=None, out=None,
+                   stream=None):
+    """gattn_decode_noalloc: the decode step without a workspace (library-held scratch)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    if v_cache is not None:
+        _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Lmax = k_cache.shape[0], k_cache.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    _raise_if(lib().gattn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(out),
+                                         B, Lmax, ctypes.byref(layer.cfg), _stream(stream)),
+              "gattn_decode_noalloc")
+    return out
 
 
 def check(workspace: torch.Tensor, stream=None) -> int:

@@ -142,6 +142,33 @@ int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf1
                  const int32_t* seq_lens, gattn_bf16* out, int32_t batch, int32_t max_len,
                  const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream);
 
+/* ---- decode without a workspace ----------------------------------------------------
+ * The model cards describe no such call; it exists for callers that cannot
+ * allocate device memory at the point where they decode: code running inside
+ * an allocator-free or pre-planned memory region (e.g. a serving loop whose
+ * pool is fixed up front), or code that must not call cudaMalloc while other
+ * work is in flight.  It computes exactly what gattn_decode computes, with the
+ * same arguments minus the workspace, and calls no cudaMalloc, cudaFree or any
+ * allocating routine.
+ * Its split partials live in a 16 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits.  The first
+ * call on each device looks up that array's device address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture.  Calls share the array: two calls whose work overlaps on
+ * the GPU (different streams, or different host threads on one device) race
+ * and may return wrong results; order them on one stream.  Nothing in the
+ * array needs to start at zero (every partial is written before it is read),
+ * and it keeps the last call's partials.
+ * If batch * num_heads * (head_dim + 2) * 4 bytes exceed the array, it returns
+ * GATTN_ERR_UNSUPPORTED and enqueues nothing; otherwise it uses fewer, longer
+ * splits when the normal split count would not fit.  There is no status word,
+ * so kernel-side range errors (a seq_lens entry outside [1, max_len], a
+ * position past the RoPE table) are not reported: such rows are written as
+ * zeros / clamped exactly as gattn_decode does. */
+int gattn_decode_noalloc(const gattn_bf16* q, const gattn_bf16* k_cache,
+                         const gattn_bf16* v_cache_or_null, const int32_t* seq_lens, gattn_bf16* out,
+                         int32_t batch, int32_t max_len, const gattn_cfg* cfg, gattn_stream stream);
+
 /* ---- status --------------------------------------------------------------------
  * gattn_check synchronises `stream`, reads and clears the workspace status
  * word, and returns GATTN_ERR_TIMEOUT or GATTN_ERR_DEVICE_BOUNDS if a kernel
