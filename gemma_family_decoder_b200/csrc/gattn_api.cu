@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -87,6 +88,10 @@ int resolve(const gattn_cfg* cfg, gattn::LayerArgs* la, bool need_ptrs) {
   la->rot = R;
   la->rope_max_pos = cfg->rope_max_pos;
   la->rope_tab = reinterpret_cast<const float2*>(cfg->rope_table);
+  la->rope_turns = (R > 0 && cfg->rope_table)
+                       ? reinterpret_cast<const double*>(cfg->rope_table +
+                                                         static_cast<size_t>(cfg->rope_max_pos) * R)
+                       : nullptr;
   la->softcap = cfg->softcap;
   la->scale = 1.0f / std::sqrt(cfg->scalar);
   la->scale_log2 = la->scale * 1.4426950408889634f;
@@ -194,7 +199,8 @@ void gattn_set_wait_timeout_us(uint32_t timeout_us) {
 
 size_t gattn_rope_table_bytes(int32_t max_pos, int32_t rot_dim) {
   if (max_pos <= 0 || rot_dim <= 0 || (rot_dim & 1)) return 0;
-  return static_cast<size_t>(max_pos) * (rot_dim / 2) * 2 * sizeof(float);
+  return static_cast<size_t>(max_pos) * (rot_dim / 2) * 2 * sizeof(float) +
+         static_cast<size_t>(rot_dim / 2) * sizeof(double);
 }
 
 int gattn_rope_table_fill(float* table, float theta, int32_t rot_dim, int32_t freq_dim,
@@ -282,8 +288,9 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   pa.trace = static_cast<unsigned long long*>(g_trace_buf);
   pa.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
-  cudaError_t e = gattn::prefill_pair_supported(la) ? gattn::launch_prefill_pair(pa, la, s)
-                                                    : gattn::launch_prefill(pa, la, s);
+  static const bool pair_off = getenv("GATTN_NO_PAIR") != nullptr;  // temporary A/B knob
+  cudaError_t e = (!pair_off && gattn::prefill_pair_supported(la)) ? gattn::launch_prefill_pair(pa, la, s)
+                                                                  : gattn::launch_prefill(pa, la, s);
   if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
   if (e != cudaSuccess) return fail_cuda(e, "prefill launch");
   return GATTN_OK;

@@ -345,6 +345,18 @@ __device__ __forceinline__ float tanh_fast(float x) {
   return y;
 }
 
+// (cos, sin) of the RoPE angle pos * theta^(-2t/F), given the angle of one
+// position step in turns (theta^(-2t/F) / 2pi): the product is formed and
+// reduced to [-1/2, 1/2] turns in double precision, then the hardware sine and
+// cosine run on an argument in [-pi, pi], where they are accurate to ~4e-7.
+__device__ __forceinline__ float2 rope_cos_sin(int pos, double turns_per_step) {
+  const double x = static_cast<double>(pos) * turns_per_step;
+  const float r = static_cast<float>(x - rint(x));
+  float s, c;
+  __sincosf(r * 6.28318530717958647692f, &s, &c);
+  return make_float2(c, s);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

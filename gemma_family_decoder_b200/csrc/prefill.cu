@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           flag_status(P.status, kStatusBounds);
           pos = pos < 0 ? 0 : la.rope_max_pos - 1;
         }
-        const float4* trow = reinterpret_cast<const float4*>(la.rope_tab + static_cast<size_t>(pos) * (la.rot >> 1));
+        const double2* turns2 = reinterpret_cast<const double2*>(la.rope_turns);
 #pragma unroll 2
         for (int c = 0; c < h8; ++c) {
           float x[8], y[8];
@@ -251,18 +251,16 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           unpack8(*chunk(c + h8), y);
           gain8(c, x);
           gain8(c + h8, y);
-          float cs[16];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 f = __ldg(trow + 4 * c + v);
-            cs[4 * v] = f.x; cs[4 * v + 1] = f.y; cs[4 * v + 2] = f.z; cs[4 * v + 3] = f.w;
-          }
           float xo[8], yo[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float co = cs[2 * e], si = cs[2 * e + 1];
-            xo[e] = x[e] * co - y[e] * si;
-            yo[e] = y[e] * co + x[e] * si;
+          for (int v = 0; v < 4; ++v) {
+            // angles of pairs 8c+2v, 8c+2v+1 computed here: no table reads
+            const double2 tv = __ldg(turns2 + 4 * c + v);
+            const float2 c0 = rope_cos_sin(pos, tv.x), c1 = rope_cos_sin(pos, tv.y);
+            xo[2 * v] = x[2 * v] * c0.x - y[2 * v] * c0.y;
+            yo[2 * v] = y[2 * v] * c0.x + x[2 * v] * c0.y;
+            xo[2 * v + 1] = x[2 * v + 1] * c1.x - y[2 * v + 1] * c1.y;
+            yo[2 * v + 1] = y[2 * v + 1] * c1.x + x[2 * v + 1] * c1.y;
           }
           *chunk(c) = pack8(xo);
           *chunk(c + h8) = pack8(yo);

@@ -24,6 +24,12 @@ using bf16 = __nv_bfloat16;
 __global__ void rope_table_kernel(float2* tab, double theta, int half, int freq_dim,
                                   long long total) {
   long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  if (i < half) {
+    // after the (cos, sin) rows: the angle of one position step in turns
+    double* turns = reinterpret_cast<double*>(tab + total);
+    turns[i] = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(freq_dim)) /
+               6.283185307179586476925286766559;
+  }
   if (i >= total) return;
   const int p = static_cast<int>(i / half);
   const int t = static_cast<int>(i % half);

@@ -120,10 +120,17 @@ def test_mqa_equals_replicated_gqa_on_gpu():
     base = W.Layer(num_heads=8, num_kv_heads=1, head_dim=256, window=50)
     d = small_prefill_inputs(base, 1, 160, seed=8)
     out_mqa, _ = run_prefill(d)
-    rep = dict(d, k=d["k"].repeat(1, 1, 8, 1), v=d["v"].repeat(1, 1, 8, 1),
-               layer=dataclasses.replace(base, num_kv_heads=8))
-    out_rep, _ = run_prefill(rep)
-    assert torch.equal(out_mqa, out_rep)
+    for hkv in (2, 4, 8):
+        rep = dict(d, k=d["k"].repeat(1, 1, hkv, 1), v=d["v"].repeat(1, 1, hkv, 1),
+                   layer=dataclasses.replace(base, num_kv_heads=hkv))
+        out_rep, _ = run_prefill(rep)
+        if hkv < 8:
+            # same kernel (query heads in pairs), same arithmetic: bit-identical
+            assert torch.equal(out_mqa, out_rep), hkv
+        else:
+            # one head per group runs the single-SM kernel: equal to rounding
+            mx, mean = err_stats(out_rep, out_mqa.double().cpu().numpy())
+            assert mx <= 1e-2 and mean <= 1e-3
 
 
 # --- the workloads at full size ---------------------------------------------------
