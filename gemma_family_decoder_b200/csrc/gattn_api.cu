@@ -88,10 +88,8 @@ int resolve(const gattn_cfg* cfg, gattn::LayerArgs* la, bool need_ptrs) {
   la->rot = R;
   la->rope_max_pos = cfg->rope_max_pos;
   la->rope_tab = reinterpret_cast<const float2*>(cfg->rope_table);
-  la->rope_turns = (R > 0 && cfg->rope_table)
-                       ? reinterpret_cast<const double*>(cfg->rope_table +
-                                                         static_cast<size_t>(cfg->rope_max_pos) * R)
-                       : nullptr;
+  la->rope_ratio = std::pow(static_cast<double>(cfg->rope_theta),
+                            -2.0 / static_cast<double>(cfg->rope_freq_dim ? cfg->rope_freq_dim : D));
   la->softcap = cfg->softcap;
   la->scale = 1.0f / std::sqrt(cfg->scalar);
   la->scale_log2 = la->scale * 1.4426950408889634f;
@@ -199,8 +197,7 @@ void gattn_set_wait_timeout_us(uint32_t timeout_us) {
 
 size_t gattn_rope_table_bytes(int32_t max_pos, int32_t rot_dim) {
   if (max_pos <= 0 || rot_dim <= 0 || (rot_dim & 1)) return 0;
-  return static_cast<size_t>(max_pos) * (rot_dim / 2) * 2 * sizeof(float) +
-         static_cast<size_t>(rot_dim / 2) * sizeof(double);
+  return static_cast<size_t>(max_pos) * (rot_dim / 2) * 2 * sizeof(float);
 }
 
 int gattn_rope_table_fill(float* table, float theta, int32_t rot_dim, int32_t freq_dim,

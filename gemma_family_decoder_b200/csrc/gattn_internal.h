@@ -18,7 +18,7 @@ struct LayerArgs {
   int rot;             // rotated dims R (0, or a power of two multiple of 16, <= D)
   int rope_max_pos;
   const float2* rope_tab;  // [max_pos][R/2] (cos, sin)
-  const double* rope_turns;  // [R/2] theta^(-2t/F) / (2 pi): turns per position step
+  double rope_ratio;      // theta^(-2/F): pair t turns theta^(-2t/F) = rope_ratio^t per position
   float softcap;       // 0 = off
   float scale_log2;    // scalar^-1/2 * log2(e)
   float scale;         // scalar^-1/2

@@ -1,0 +1,203 @@
+// Warp-per-row helpers for the QK-norm + RoPE prologue (sm_100a).
+//
+// A warp holds one head row of D = 256 * NCH dims; lane l owns the 8-dim
+// chunks c = l + 32 i (i < NCH), dims [8c, 8c + 8).  Used by the key prologue,
+// the decode query/key prologues and the prefill query prologue.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "gattn_internal.h"
+#include "kernels/common.cuh"
+
+namespace gattn {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int NCH>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* row, int lane, float (&x)[NCH][8]) {
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + lane + 32 * i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(w[e]);
+      x[i][2 * e] = f.x;
+      x[i][2 * e + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ int checked_pos(int pos, const LayerArgs& la, uint32_t* status) {
+  if (pos < 0 || pos >= la.rope_max_pos) {
+    flag_status(status, kStatusBounds);
+    return pos < 0 ? 0 : la.rope_max_pos - 1;
+  }
+  return pos;
+}
+
+// RMSNorm (optional) then RoPE (optional) on a warp-held row, in fp32.
+template <int NCH>
+__device__ __forceinline__ void transform_row(float (&x)[NCH][8], int lane, int pos,
+                                              const LayerArgs& la, const float* w,
+                                              uint32_t* status) {
+  constexpr int D = NCH * 256;
+  if (la.qk_norm) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += x[i][e] * x[i][e];
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+    const float off = la.qk_norm == 1 ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int d = 8 * (lane + 32 * i) + e;
+        x[i][e] = x[i][e] * r * (__ldg(w + d) + off);
+      }
+  }
+  if (la.rot > 0) {
+    pos = checked_pos(pos, la, status);
+    const int half = la.rot >> 1;
+    const int h16 = la.rot >> 4;  // chunks in half the rotated slice
+    float pr[NCH][8];
+    if (h16 < 32) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = __shfl_xor_sync(0xffffffffu, x[i][e], h16);
+    } else {
+      // rotated slice of 512 dims: the partner chunk is this lane's other chunk
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = x[NCH - 1 - i][e];
+    }
+    const float2* trow = la.rope_tab + static_cast<size_t>(pos) * half;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = lane + 32 * i;
+      if (8 * c < la.rot) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int d = 8 * c + e;
+          const bool first = d < half;
+          const float2 cs = __ldg(trow + (first ? d : d - half));
+          x[i][e] = first ? x[i][e] * cs.x - pr[i][e] * cs.y : x[i][e] * cs.x + pr[i][e] * cs.y;
+        }
+      }
+    }
+  }
+}
+
+
+// 8 floats <-> 8 packed bf16 (16 bytes)
+__device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = unpack_bf16x2(w[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]);
+  u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]);
+  u.w = pack_bf16x2(x[6], x[7]);
+  return u;
+}
+
+// Query prologue of a prefill tile held in shared memory (128 rows, 128-byte
+// swizzled 64-dim slabs), in place, on one row: RMSNorm over the row, then RoPE
+// with angles computed here (pair t turns theta^(-2t/F) / 2pi per position,
+// built as a geometric sequence in double precision), so the only global read
+// is the row's position.  A row may be split between threads: tile_row_sumsq
+// gives the partial sum of squares of chunks [c_lo, c_hi), and
+// tile_row_prologue rotates the pair chunks [pc_lo, pc_hi) (chunk c with chunk
+// c + R/16) and scales the unrotated chunks [uc_lo, uc_hi) by the norm.
+__device__ __forceinline__ uint4* tile_chunk(uint8_t* tile, int slab_bytes, int r, int c) {
+  return reinterpret_cast<uint4*>(tile + (c >> 3) * slab_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ float tile_row_sumsq(uint8_t* tile, int slab_bytes, int r, int c_lo,
+                                                int c_hi) {
+  float ss = 0.f;
+#pragma unroll 4
+  for (int c = c_lo; c < c_hi; ++c) {
+    float x[8];
+    unpack8(*tile_chunk(tile, slab_bytes, r, c), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+  }
+  return ss;
+}
+
+// rn: 1/rms of the whole row (ignored without QK-norm).
+__device__ __forceinline__ void tile_row_prologue(uint8_t* tile, int slab_bytes, int r, int pos,
+                                                  const LayerArgs& la, float rn, int pc_lo,
+                                                  int pc_hi, int uc_lo, int uc_hi) {
+  const float off = la.qk_norm == 1 ? 1.f : 0.f;
+  const float4* g4 = reinterpret_cast<const float4*>(la.q_norm_w);
+  auto gain8 = [&](int c, float (&x)[8]) {
+    if (!la.qk_norm) return;
+    const float4 g0 = __ldg(g4 + 2 * c), g1 = __ldg(g4 + 2 * c + 1);
+    x[0] *= rn * (g0.x + off); x[1] *= rn * (g0.y + off);
+    x[2] *= rn * (g0.z + off); x[3] *= rn * (g0.w + off);
+    x[4] *= rn * (g1.x + off); x[5] *= rn * (g1.y + off);
+    x[6] *= rn * (g1.z + off); x[7] *= rn * (g1.w + off);
+  };
+  const int h8 = la.rot >> 4;  // 8-dim chunks in half the rotated slice
+  if (la.rot > 0 && pc_lo < pc_hi) {
+    const double q = la.rope_ratio;
+    double qp[8];  // q^e, e < 8
+    qp[0] = 1.0;
+#pragma unroll
+    for (int e = 1; e < 8; ++e) qp[e] = qp[e - 1] * q;
+    const double q8 = qp[7] * q;
+    double f8 = 0.15915494309189533576888376337251;  // turns per radian: pair 0
+    for (int c = 0; c < pc_lo; ++c) f8 *= q8;
+#pragma unroll 2
+    for (int c = pc_lo; c < pc_hi; ++c) {
+      uint4* cx = tile_chunk(tile, slab_bytes, r, c);
+      uint4* cy = tile_chunk(tile, slab_bytes, r, c + h8);
+      float x[8], y[8];
+      unpack8(*cx, x);
+      unpack8(*cy, y);
+      gain8(c, x);
+      gain8(c + h8, y);
+      float xo[8], yo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float2 cs = rope_cos_sin(pos, f8 * qp[e]);
+        xo[e] = x[e] * cs.x - y[e] * cs.y;
+        yo[e] = y[e] * cs.x + x[e] * cs.y;
+      }
+      *cx = pack8(xo);
+      *cy = pack8(yo);
+      f8 *= q8;
+    }
+  }
+  if (la.qk_norm) {
+#pragma unroll 4
+    for (int c = uc_lo; c < uc_hi; ++c) {
+      uint4* cx = tile_chunk(tile, slab_bytes, r, c);
+      float x[8];
+      unpack8(*cx, x);
+      gain8(c, x);
+      *cx = pack8(x);
+    }
+  }
+}
+
+}  // namespace gattn

@@ -27,6 +27,7 @@
 
 #include "gattn_internal.h"
 #include "kernels/common.cuh"
+#include "kernels/rowops.cuh"
 
 namespace gattn {
 
@@ -128,6 +129,11 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   const int kv_lo = la.window > 0 ? max(0, q0 - la.window + 1) : 0;
   const int k_first = (kv_lo / BN) * BN;
   const int ntiles = (kv_hi - k_first + BN - 1) / BN;
+  // KV tiles are visited starting at a tile that differs between the CTAs
+  // working on one sequence at once, so they do not all read the same L2 lines
+  // together (the online softmax is independent of the visiting order)
+  const int rot = ntiles > 1 ? (h * 7 + dvs * 3 + b * 5 + qt) % ntiles : 0;
+  auto tile_key = [&](int j) { return k_first + ((j + rot) % ntiles) * BN; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -192,89 +198,17 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     }
 
     // query prologue in place: RMSNorm + RoPE in fp32 on this thread's row
+    // query prologue in place, thread t on row t; RoPE angles computed, not read
     if (ok && valid && (la.rot > 0 || la.qk_norm)) {
-      uint8_t* qrow = smem + C::OFF_Q + t * 128;
-      auto chunk = [&](int c) -> uint4* {
-        return reinterpret_cast<uint4*>(qrow + (c >> 3) * C::SLAB128 + (((c & 7) ^ (t & 7)) << 4));
-      };
-      auto unpack8 = [](uint4 u, float (&x)[8]) {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_bf16x2(w[e]);
-          x[2 * e] = f.x;
-          x[2 * e + 1] = f.y;
-        }
-      };
-      auto pack8 = [](const float (&x)[8]) {
-        uint4 u;
-        u.x = pack_bf16x2(x[0], x[1]);
-        u.y = pack_bf16x2(x[2], x[3]);
-        u.z = pack_bf16x2(x[4], x[5]);
-        u.w = pack_bf16x2(x[6], x[7]);
-        return u;
-      };
-      float r = 1.f;
-      if (la.qk_norm) {
-        float ss = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < D / 8; ++c) {
-          float x[8];
-          unpack8(*chunk(c), x);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-        }
-        r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+      int pos = la.rot > 0 ? __ldg(P.positions + static_cast<size_t>(b) * S + qi) : 0;
+      if (la.rot > 0 && (pos < 0 || pos >= la.rope_max_pos)) {
+        flag_status(P.status, kStatusBounds);
+        pos = pos < 0 ? 0 : la.rope_max_pos - 1;
       }
-      const float off = la.qk_norm == 1 ? 1.f : 0.f;
-      const float4* g4 = reinterpret_cast<const float4*>(la.q_norm_w);
-      auto gain8 = [&](int c, float (&x)[8]) {
-        if (!la.qk_norm) return;
-        const float4 g0 = __ldg(g4 + 2 * c), g1 = __ldg(g4 + 2 * c + 1);
-        x[0] *= r * (g0.x + off); x[1] *= r * (g0.y + off);
-        x[2] *= r * (g0.z + off); x[3] *= r * (g0.w + off);
-        x[4] *= r * (g1.x + off); x[5] *= r * (g1.y + off);
-        x[6] *= r * (g1.z + off); x[7] *= r * (g1.w + off);
-      };
-      const int h8 = la.rot >> 4;  // chunks in half the rotated slice
-      if (la.rot > 0) {
-        int pos = __ldg(P.positions + static_cast<size_t>(b) * S + qi);
-        if (pos < 0 || pos >= la.rope_max_pos) {
-          flag_status(P.status, kStatusBounds);
-          pos = pos < 0 ? 0 : la.rope_max_pos - 1;
-        }
-        const double2* turns2 = reinterpret_cast<const double2*>(la.rope_turns);
-#pragma unroll 2
-        for (int c = 0; c < h8; ++c) {
-          float x[8], y[8];
-          unpack8(*chunk(c), x);
-          unpack8(*chunk(c + h8), y);
-          gain8(c, x);
-          gain8(c + h8, y);
-          float xo[8], yo[8];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            // angles of pairs 8c+2v, 8c+2v+1 computed here: no table reads
-            const double2 tv = __ldg(turns2 + 4 * c + v);
-            const float2 c0 = rope_cos_sin(pos, tv.x), c1 = rope_cos_sin(pos, tv.y);
-            xo[2 * v] = x[2 * v] * c0.x - y[2 * v] * c0.y;
-            yo[2 * v] = y[2 * v] * c0.x + x[2 * v] * c0.y;
-            xo[2 * v + 1] = x[2 * v + 1] * c1.x - y[2 * v + 1] * c1.y;
-            yo[2 * v + 1] = y[2 * v + 1] * c1.x + x[2 * v + 1] * c1.y;
-          }
-          *chunk(c) = pack8(xo);
-          *chunk(c + h8) = pack8(yo);
-        }
-      }
-      if (la.qk_norm) {
-#pragma unroll 4
-        for (int c = 2 * h8; c < D / 8; ++c) {
-          float x[8];
-          unpack8(*chunk(c), x);
-          gain8(c, x);
-          *chunk(c) = pack8(x);
-        }
-      }
+      const float rn = la.qk_norm ? rsqrtf(tile_row_sumsq(smem + C::OFF_Q, C::SLAB128, t, 0, D / 8) /
+                                               static_cast<float>(D) + la.eps)
+                                  : 1.f;
+      tile_row_prologue(smem + C::OFF_Q, C::SLAB128, t, pos, la, rn, 0, la.rot >> 4, la.rot >> 3, D / 8);
     }
     if constexpr (QTM) {
       // move this thread's row into the Q columns of TMEM (64 dims per x32 store)
@@ -317,7 +251,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
       tmem_wait_ld();
 
-      const int key0 = k_first + j * BN;
+      const int key0 = tile_key(j);
       const bool full_tile = (key0 + BN - 1 <= q0) && (q0 + C::BM <= S) &&
                              (W <= 0 || (q0 + C::BM - 1) - key0 < W);
       float x[BN];
@@ -455,11 +389,11 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       // same order as the MMA issuer consumes them: K(j) then V(j-1)
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
-        const int key0 = k_first + j * BN;
+        const int key0 = tile_key(j);
         for (int c = 0; c < C::KCH && ok; ++c) ok = load(&P.tm_k, c * 64, key0);
-        for (int c = 0; c < C::VCH && ok && j >= 1; ++c) ok = load(&P.tm_v, dv_lo + c * 64, key0 - BN);
+        for (int c = 0; c < C::VCH && ok && j >= 1; ++c) ok = load(&P.tm_v, dv_lo + c * 64, tile_key(j - 1));
       }
-      for (int c = 0; c < C::VCH && ok; ++c) ok = load(&P.tm_v, dv_lo + c * 64, k_first + (ntiles - 1) * BN);
+      for (int c = 0; c < C::VCH && ok; ++c) ok = load(&P.tm_v, dv_lo + c * 64, tile_key(ntiles - 1));
       // let every issued copy land before the CTA can exit
       if constexpr (!QTM) mbar_wait(q_full, 0, tmo, P.status, nullptr);
       for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)

@@ -7,18 +7,21 @@
 // shared memory (keys [0,64) / [64,128) of a key tile for Q K^T, value dims
 // [0,128) / [128,256) for P V), so each SM loads half of the K/V bytes a
 // single-SM tile would.  Roles per CTA:
-//   warps 0-3  Q-tile prologue (QK-norm + RoPE in place in shared memory), then
-//              per KV tile the online softmax on this CTA's S rows in TMEM, P
-//              written back over its S slot, and the O / l epilogue + TMA store.
-//   warp 4     TMA producer for this CTA's Q tile and K/V halves; ring-slot
+//   warps 0-7  two threads per query row (warp w: TMEM lanes 32*(w%4).., column
+//              half w/4): Q-tile prologue (QK-norm + RoPE in place in shared
+//              memory), then per KV tile the online softmax on this CTA's S rows
+//              (the halves exchange only the row maximum), P written back over
+//              its S slot, and the O / l epilogue + TMA store.
+//   warp 8     TMA producer for this CTA's Q tile and K/V halves; ring-slot
 //              completion is counted on the barriers of CTA 0.
-//   warp 5     (CTA 0 only) issues the pair MMAs and their commits, which arrive
+//   warp 9     (CTA 0 only) issues the pair MMAs and their commits, which arrive
 //              on the matching barriers of both CTAs.
 // The layer definition is the one of the single-SM kernel (prefill.cu).
 #include <cuda_bf16.h>
 
 #include "gattn_internal.h"
 #include "kernels/common.cuh"
+#include "kernels/rowops.cuh"
 
 namespace gattn {
 
@@ -38,12 +41,13 @@ struct PairShape {
   static constexpr int VBOX = BN * 128;          // 64 dims x 128 keys
   static constexpr int KSLOTS = 2;               // this CTA's key half: 4 boxes of 8 KB
   static constexpr int VSLOTS = 2;               // this CTA's value half: 2 boxes of 16 KB
-  static constexpr int NSTAGE = 10;              // even: 2-slot units never wrap
+  static constexpr int NSTAGE = 8;               // even: 2-slot units never wrap
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = Q_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * SLOT;
   static constexpr int NBAR = 2 * NSTAGE + 12;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_XCH = OFF_BAR + NBAR * 8;     // row exchange: 2 x 256 floats
+  static constexpr int OFF_MISC = OFF_XCH + 512 * 4;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TM_O = 0;
   static constexpr uint32_t TM_S0 = DV;
@@ -64,6 +68,8 @@ struct PairParams {
   uint64_t timeout_ns;
   int B, S, nqt, pairs_per_group;
   LayerArgs la;
+  unsigned long long* trace;  // optional per-CTA timeline (same slots as the single-SM kernel)
+  int trace_ctas;
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -71,7 +77,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace
 
 template <bool CAP>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     prefill_pair_kernel(const __grid_constant__ PairParams P) {
   using C = PairShape;
   extern __shared__ uint8_t smem_raw[];
@@ -81,9 +87,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* full = bars;                     // CTA 0's copy counts both CTAs' bytes
   uint64_t* empty = bars + C::NSTAGE;        // both CTAs (multicast commits)
   uint64_t* s_full = bars + 2 * C::NSTAGE;   // [2], both CTAs
-  uint64_t* p_full = s_full + 2;             // [2], CTA 0: 256 arrivals
+  uint64_t* p_full = s_full + 2;             // [2], CTA 0: 512 arrivals
   uint64_t* o_done = p_full + 2;             // both CTAs
-  uint64_t* q_ready = o_done + 1;            // CTA 0: 256 arrivals
+  uint64_t* q_ready = o_done + 1;            // CTA 0: 512 arrivals
   uint64_t* drain = q_ready + 1;             // CTA 0
   uint64_t* q_full = drain + 1;              // own Q tile
   uint64_t* o_final = q_full + 1;            // both CTAs
@@ -108,6 +114,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const int kv_lo = la.window > 0 ? max(0, q0 - la.window + 1) : 0;
   const int k_first = (kv_lo / C::BN) * C::BN;
   const int ntiles = (kv_hi - k_first + C::BN - 1) / C::BN;
+  // KV tiles are visited starting at a tile that differs between the pairs
+  // working on one sequence at once, so they do not all read the same L2 lines
+  // together (the online softmax is independent of the visiting order)
+  const int rot = ntiles > 1 ? (pg * 7 + kvh * 3 + b * 5 + qt) % ntiles : 0;
+  auto tile_key = [&](int j) { return k_first + ((j + rot) % ntiles) * C::BN; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -117,23 +128,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
+      mbar_init(&p_full[i], 512);
     }
     mbar_init(o_done, 1);
-    mbar_init(q_ready, 256);
+    mbar_init(q_ready, 512);
     mbar_init(drain, 1);
     mbar_init(q_full, 1);
     mbar_init(o_final, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&P.tm_q);
     tma_prefetch_desc(&P.tm_k);
     tma_prefetch_desc(&P.tm_v);
     tma_prefetch_desc(&P.tm_o);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
@@ -142,140 +153,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = P.timeout_ns;
+  unsigned long long* trace = (P.trace && static_cast<int>(blockIdx.x) < P.trace_ctas)
+                                  ? P.trace + static_cast<size_t>(blockIdx.x) * 512 : nullptr;
+  const uint64_t t_start = globaltimer_ns();
+  auto mark = [&](int slot) {
+    if (trace) trace[slot] = globaltimer_ns() - t_start;
+  };
+  if (trace && threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    trace[0] = t_start;
+    trace[1] = smid;
+    trace[2] = ntiles;
+  }
   // CTA 0's copies of the barriers that count both CTAs
   auto leader = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------------ softmax
+    // two threads per query row: warp w reads TMEM lanes 32*(w%4).. and owns
+    // the key / value-dim half hf = w / 4 of every tile
+    const int r = (warp & 3) * 32 + lane;     // query row of this thread
+    const int hf = warp >> 2;                 // column half
     const int t = threadIdx.x;
-    const int qi = q0 + t;
+    const int qi = q0 + r;
     const bool valid = qi < S;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // row exchange between the two halves, [2 regions][2 halves][128 rows]: the
+    // norm sums use region 1, tile j's maxima region j&1, the final sums region
+    // ntiles&1, so no region is rewritten while a slower thread may still read it
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
-    if (ok && valid && (la.rot > 0 || la.qk_norm)) {
-      uint8_t* qrow = smem + C::OFF_Q + t * 128;
-      auto chunk = [&](int c) -> uint4* {
-        return reinterpret_cast<uint4*>(qrow + (c >> 3) * C::SLAB128 + (((c & 7) ^ (t & 7)) << 4));
-      };
-      auto unpack8 = [](uint4 u, float (&x)[8]) {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_bf16x2(w[e]);
-          x[2 * e] = f.x;
-          x[2 * e + 1] = f.y;
-        }
-      };
-      auto pack8 = [](const float (&x)[8]) {
-        uint4 u;
-        u.x = pack_bf16x2(x[0], x[1]);
-        u.y = pack_bf16x2(x[2], x[3]);
-        u.z = pack_bf16x2(x[4], x[5]);
-        u.w = pack_bf16x2(x[6], x[7]);
-        return u;
-      };
-      float r = 1.f;
+    if (t == 0) mark(6);
+    // query prologue in place; RoPE angles computed, not read
+    {
+      const int h8 = la.rot >> 4, nu = C::D / 8 - 2 * h8;
+      float rn = 1.f;
       if (la.qk_norm) {
-        float ss = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < C::D / 8; ++c) {
-          float x[8];
-          unpack8(*chunk(c), x);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-        }
-        r = rsqrtf(ss / static_cast<float>(C::D) + la.eps);
+        const float ss = (ok && valid) ? tile_row_sumsq(smem + C::OFF_Q, C::SLAB128, r, hf * (C::D / 16),
+                                                        (hf + 1) * (C::D / 16))
+                                       : 0.f;
+        xch[256 + hf * 128 + r] = ss;
+        named_barrier(1, 256);
+        rn = rsqrtf((xch[256 + r] + xch[256 + 128 + r]) / static_cast<float>(C::D) + la.eps);
       }
-      const float off = la.qk_norm == 1 ? 1.f : 0.f;
-      const float4* g4 = reinterpret_cast<const float4*>(la.q_norm_w);
-      auto gain8 = [&](int c, float (&x)[8]) {
-        if (!la.qk_norm) return;
-        const float4 g0 = __ldg(g4 + 2 * c), g1 = __ldg(g4 + 2 * c + 1);
-        x[0] *= r * (g0.x + off); x[1] *= r * (g0.y + off);
-        x[2] *= r * (g0.z + off); x[3] *= r * (g0.w + off);
-        x[4] *= r * (g1.x + off); x[5] *= r * (g1.y + off);
-        x[6] *= r * (g1.z + off); x[7] *= r * (g1.w + off);
-      };
-      const int h8 = la.rot >> 4;
-      if (la.rot > 0) {
-        int pos = __ldg(P.positions + static_cast<size_t>(b) * S + qi);
-        if (pos < 0 || pos >= la.rope_max_pos) {
+      if (ok && valid && (la.rot > 0 || la.qk_norm)) {
+        int pos = la.rot > 0 ? __ldg(P.positions + static_cast<size_t>(b) * S + qi) : 0;
+        if (la.rot > 0 && (pos < 0 || pos >= la.rope_max_pos)) {
           flag_status(P.status, kStatusBounds);
           pos = pos < 0 ? 0 : la.rope_max_pos - 1;
         }
-        const double2* turns2 = reinterpret_cast<const double2*>(la.rope_turns);
-#pragma unroll 2
-        for (int c = 0; c < h8; ++c) {
-          float x[8], y[8];
-          unpack8(*chunk(c), x);
-          unpack8(*chunk(c + h8), y);
-          gain8(c, x);
-          gain8(c + h8, y);
-          float xo[8], yo[8];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            // angles of pairs 8c+2v, 8c+2v+1 computed here: no table reads
-            const double2 tv = __ldg(turns2 + 4 * c + v);
-            const float2 c0 = rope_cos_sin(pos, tv.x), c1 = rope_cos_sin(pos, tv.y);
-            xo[2 * v] = x[2 * v] * c0.x - y[2 * v] * c0.y;
-            yo[2 * v] = y[2 * v] * c0.x + x[2 * v] * c0.y;
-            xo[2 * v + 1] = x[2 * v + 1] * c1.x - y[2 * v + 1] * c1.y;
-            yo[2 * v + 1] = y[2 * v + 1] * c1.x + x[2 * v + 1] * c1.y;
-          }
-          *chunk(c) = pack8(xo);
-          *chunk(c + h8) = pack8(yo);
-        }
-      }
-      if (la.qk_norm) {
-#pragma unroll 4
-        for (int c = 2 * h8; c < C::D / 8; ++c) {
-          float x[8];
-          unpack8(*chunk(c), x);
-          gain8(c, x);
-          *chunk(c) = pack8(x);
-        }
+        tile_row_prologue(smem + C::OFF_Q, C::SLAB128, r, pos, la, rn, (hf * h8) >> 1, ((hf + 1) * h8) >> 1,
+                          2 * h8 + ((hf * nu) >> 1), 2 * h8 + (((hf + 1) * nu) >> 1));
       }
     }
     fence_proxy_async_smem();
     mbar_arrive_cluster(leader(q_ready));
+    if (t == 0) mark(7);
 
     const float sl2 = la.scale_log2;
     const float kcap = CAP ? la.scale / la.softcap : 0.f;
     const float cap_l2 = CAP ? la.softcap * kLog2e : 0.f;
     const int W = la.window;
-    float m = -INFINITY, l = 0.f;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag));
-      if (!ok) break;
+    constexpr int HN = C::BN / 2;            // keys per thread per tile
+    float m = -INFINITY, l = 0.f;            // l: this thread's half of the row sum
+    // every thread reaches the per-tile barrier each iteration; the loop is left
+    // by all 256 at once when any wait has failed
+    for (int j = 0; j < ntiles; ++j) {
+      const bool got = ok && mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag);
+      if (t == 0 && j < 60) mark(8 + j);
       tc_fence_after();
       const uint32_t scol = tmem + lane_off + ((j & 1) ? C::TM_S1 : C::TM_S0);
-      uint32_t rr[C::BN / 32][32];
+      uint32_t rr[HN / 32][32];
 #pragma unroll
-      for (int c = 0; c < C::BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
+      for (int c = 0; c < HN / 32; ++c) tmem_ld32(scol + hf * HN + c * 32, rr[c]);
       tmem_wait_ld();
 
-      const int key0 = k_first + j * C::BN;
-      const bool full_tile = (key0 + C::BN - 1 <= q0) && (q0 + C::BM <= S) &&
-                             (W <= 0 || (q0 + C::BM - 1) - key0 < W);
-      float x[C::BN];
+      const int tkey0 = tile_key(j);
+      const int key0 = tkey0 + hf * HN;   // first key of this thread's half
+      const bool full_tile = (tkey0 + C::BN - 1 <= q0) && (q0 + C::BM <= S) &&
+                             (W <= 0 || (q0 + C::BM - 1) - tkey0 < W);
+      float x[HN];
 #pragma unroll
-      for (int i = 0; i < C::BN; ++i) {
-        const float s = __uint_as_float(rr[i >> 5][i & 31]);
-        x[i] = CAP ? cap_l2 * tanh_fast(s * kcap) : s;
+      for (int i = 0; i < HN; ++i) {
+        const float sv = __uint_as_float(rr[i >> 5][i & 31]);
+        x[i] = CAP ? cap_l2 * tanh_fast(sv * kcap) : sv;
       }
       if (!full_tile) {
         const int hi = valid ? qi - key0 : -1;
         const int lo = W > 0 ? qi - key0 - W + 1 : -C::BN;
 #pragma unroll
-        for (int i = 0; i < C::BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
+        for (int i = 0; i < HN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
       }
       float mxa[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mxa[a] = x[a];
 #pragma unroll
-      for (int i = 8; i < C::BN; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], x[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                             fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
+      for (int i = 8; i < HN; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], x[i]);
+      float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                       fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
+      // the row maximum over both halves (the two threads must agree on m)
+      float* xm = xch + (j & 1) * 256;
+      xm[hf * 128 + r] = mx;
+      ok = named_barrier_and(1, 256, got);
+      if (!ok) break;
+      mx = fmaxf(xm[r], xm[128 + r]);
       const float m_tile = CAP ? mx : mx * sl2;
       const float m_new = fmaxf(m, m_tile);
       float alpha = 1.f;
@@ -290,31 +272,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       float rsa[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) rsa[a] = 0.f;
-      uint32_t pk[C::BN / 64][32];
+      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < C::BN; i += 2) {
+      for (int i = 0; i < HN; i += 2) {
         const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
         const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
         rsa[(i >> 1) & 7] += p0 + p1;
-        pk[i >> 6][(i >> 1) & 31] = pack_bf16x2(p0, p1);
+        pk[i >> 1] = pack_bf16x2(p0, p1);
       }
       const float rs = ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
-#pragma unroll
-      for (int c = 0; c < C::BN / 64; ++c) tmem_st32(scol + c * 32, pk[c]);
+      // P of this half: bf16 pairs over columns [hf*HN/2, hf*HN/2 + HN/2) of the S slot
+      tmem_st32(scol + hf * (HN / 2), pk);
       // seeing S(j) implies P V(j-2) is complete, so o_done's parity wait is exact
       if (__any_sync(0xffffffffu, rescale) && j >= 1) {
+        // a failed wait is carried to the next tile's barrier, where all leave together
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag));
-        if (!ok) break;
         tc_fence_after();
         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < C::DV / 32; ++c) {
+        for (int c = 0; c < C::DV / 64; ++c) {   // this thread's half of O's columns
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+          const uint32_t oc = tmem + lane_off + C::TM_O + hf * (C::DV / 2) + c * 32;
+          tmem_ld32(oc, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
+          tmem_st32(oc, o);
         }
       }
       tmem_wait_st();
@@ -322,16 +305,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       m = m_use;
       tc_fence_before();
       mbar_arrive_cluster(leader(&p_full[j & 1]));
+      if (t == 0 && j < 60) mark(68 + j);
     }
-    ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, tmo, P.status, abort_flag));
+    ok = ok && mbar_wait(o_final, 0, tmo, P.status, abort_flag);
+    // the whole row sum: this half's plus the other's
+    float* xl = xch + (ntiles & 1) * 256;
+    xl[hf * 128 + r] = l;
+    ok = named_barrier_and(1, 256, ok);
+    const float lt = xl[r] + xl[128 + r];
     if (ok) {
+      if (t == 0) mark(4);
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint8_t* orow = smem + C::OFF_Q + t * 128;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      uint8_t* orow = smem + C::OFF_Q + r * 128;
 #pragma unroll 1
-      for (int c = 0; c < C::DV / 32; ++c) {
+      for (int c = 0; c < C::DV / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+        tmem_ld32(tmem + lane_off + C::TM_O + hf * (C::DV / 2) + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -340,12 +330,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           u.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
           u.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
           u.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-          const int ch = 4 * c + v;
-          *reinterpret_cast<uint4*>(orow + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (t & 7)) << 4)) = u;
+          const int ch = hf * (C::DV / 16) + 4 * c + v;
+          *reinterpret_cast<uint4*>(orow + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (r & 7)) << 4)) = u;
         }
       }
       fence_proxy_async_smem();
-      named_barrier(1, 128);
+      named_barrier(1, 256);
       if (t == 0) {
 #pragma unroll
         for (int sl = 0; sl < C::DV / 64; ++sl)
@@ -354,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         bulk_wait_read_all();
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, C::Q_BYTES);
@@ -367,9 +357,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         return mbar_wait(&empty[st], par, tmo, P.status, abort_flag) &&
                mbar_wait(&empty[st + 1], par, tmo, P.status, abort_flag);
       };
+      int nk = 0, nv = 0;
       auto load_k = [&](int key0) -> bool {   // this CTA's 64 keys, all 256 dims
         const int st = (2 * n) % C::NSTAGE;
         if (!wait_slots(st)) return false;
+        if (nk < 60) mark(248 + nk);
+        ++nk;
         for (int s2 = 0; s2 < 2; ++s2) {
           const uint32_t lb = leader(&full[st + s2]);
           mbar_arrive_expect_tx_cluster(lb, C::SLOT);
@@ -384,6 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       auto load_v = [&](int key0) -> bool {   // all 128 keys, this CTA's 128 value dims
         const int st = (2 * n) % C::NSTAGE;
         if (!wait_slots(st)) return false;
+        if (nv < 60) mark(308 + nv);
+        ++nv;
         for (int s2 = 0; s2 < 2; ++s2) {
           const uint32_t lb = leader(&full[st + s2]);
           mbar_arrive_expect_tx_cluster(lb, C::SLOT);
@@ -395,11 +390,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       };
       bool ok = true;
       for (int j = 0; j < ntiles && ok; ++j) {
-        const int key0 = k_first + j * C::BN;
-        ok = load_k(key0);
-        if (ok && j >= 1) ok = load_v(key0 - C::BN);
+        ok = load_k(tile_key(j));
+        if (ok && j >= 1) ok = load_v(tile_key(j - 1));
       }
-      if (ok) ok = load_v(k_first + (ntiles - 1) * C::BN);
+      if (ok) ok = load_v(tile_key(ntiles - 1));
       mbar_wait(q_full, 0, tmo, P.status, nullptr);
       if (!ok) {
         // after a timed-out wait the ring barriers are not trustworthy; give
@@ -417,6 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       constexpr uint16_t both = 0x3;
       int n = 0;
       bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
+      mark(3);
       tc_fence_after();
       auto wait_full = [&](int st) -> bool {
         const uint32_t par = (n / (C::NSTAGE / 2)) & 1;
@@ -427,6 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
         const int st = (2 * n) % C::NSTAGE;
         if (!wait_full(st)) return false;
+        if (j < 60) mark(368 + j);
         tc_fence_after();
         const uint32_t kb = sbase + C::OFF_RING + st * C::SLOT;
 #pragma unroll
@@ -444,6 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         mma_commit_pair(&empty[st + 1], both);
         mma_commit_pair(&s_full[j & 1], both);
         ++n;
+        if (j < 60) mark(128 + j);
         return true;
       };
       auto pv = [&](int i) -> bool {
@@ -451,6 +448,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
         const int st = (2 * n) % C::NSTAGE;
         if (!wait_full(st)) return false;
+        if (i < 60) mark(428 + i);
         tc_fence_after();
         const uint32_t vb = sbase + C::OFF_RING + st * C::SLOT;
 #pragma unroll
@@ -463,6 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         mma_commit_pair(&empty[st + 1], both);
         mma_commit_pair(o_done, both);
         ++n;
+        if (i < 60) mark(188 + i);
         return true;
       };
       for (int j = 0; j < ntiles && ok; ++j) {
@@ -479,10 +478,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_before();
   // neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it
   cluster_sync();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) mark(5);
 }
 
 bool prefill_pair_supported(const LayerArgs& la) { return la.D == 256 && la.G % 2 == 0; }
@@ -503,6 +503,8 @@ cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cuda
   P.nqt = (pa.S + C::BM - 1) / C::BM;
   P.pairs_per_group = la.G / 2;
   P.la = la;
+  P.trace = pa.trace;
+  P.trace_ctas = static_cast<int>(pa.trace_bytes / (512 * sizeof(unsigned long long)));
   const bool cap = la.softcap > 0.f;
   auto kern = cap ? prefill_pair_kernel<true> : prefill_pair_kernel<false>;
   static bool attr_set[2] = {false, false};
@@ -512,7 +514,7 @@ cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cuda
     attr_set[cap] = true;
   }
   const long long grid = 2LL * P.nqt * pa.B * la.Hkv * P.pairs_per_group;
-  kern<<<static_cast<unsigned>(grid), 192, C::SMEM, s>>>(P);
+  kern<<<static_cast<unsigned>(grid), 320, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
 

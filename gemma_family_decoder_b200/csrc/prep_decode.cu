@@ -13,6 +13,7 @@
 
 #include "gattn_internal.h"
 #include "kernels/common.cuh"
+#include "kernels/rowops.cuh"
 
 namespace gattn {
 
@@ -24,12 +25,6 @@ using bf16 = __nv_bfloat16;
 __global__ void rope_table_kernel(float2* tab, double theta, int half, int freq_dim,
                                   long long total) {
   long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
-  if (i < half) {
-    // after the (cos, sin) rows: the angle of one position step in turns
-    double* turns = reinterpret_cast<double*>(tab + total);
-    turns[i] = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(freq_dim)) /
-               6.283185307179586476925286766559;
-  }
   if (i >= total) return;
   const int p = static_cast<int>(i / half);
   const int t = static_cast<int>(i % half);
@@ -47,96 +42,6 @@ cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim,
   rope_table_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(tab, theta, half, freq_dim,
                                                                       total);
   return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Shared row helpers: a warp holds one head row, lane l owning dims
-// [8(l+32i), 8(l+32i)+8) for i < D/256.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-template <int NCH>
-__device__ __forceinline__ void load_row(const bf16* row, int lane, float (&x)[NCH][8]) {
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + lane + 32 * i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack_bf16x2(w[e]);
-      x[i][2 * e] = f.x;
-      x[i][2 * e + 1] = f.y;
-    }
-  }
-}
-
-__device__ __forceinline__ int checked_pos(int pos, const LayerArgs& la, uint32_t* status) {
-  if (pos < 0 || pos >= la.rope_max_pos) {
-    flag_status(status, kStatusBounds);
-    return pos < 0 ? 0 : la.rope_max_pos - 1;
-  }
-  return pos;
-}
-
-// RMSNorm (optional) then RoPE (optional) on a warp-held row, in fp32.
-template <int NCH>
-__device__ __forceinline__ void transform_row(float (&x)[NCH][8], int lane, int pos,
-                                              const LayerArgs& la, const float* w,
-                                              uint32_t* status) {
-  constexpr int D = NCH * 256;
-  if (la.qk_norm) {
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < NCH; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss += x[i][e] * x[i][e];
-    ss = warp_sum(ss);
-    const float r = rsqrtf(ss / static_cast<float>(D) + la.eps);
-    const float off = la.qk_norm == 1 ? 1.f : 0.f;
-#pragma unroll
-    for (int i = 0; i < NCH; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int d = 8 * (lane + 32 * i) + e;
-        x[i][e] = x[i][e] * r * (__ldg(w + d) + off);
-      }
-  }
-  if (la.rot > 0) {
-    pos = checked_pos(pos, la, status);
-    const int half = la.rot >> 1;
-    const int h16 = la.rot >> 4;  // chunks in half the rotated slice
-    float pr[NCH][8];
-    if (h16 < 32) {
-#pragma unroll
-      for (int i = 0; i < NCH; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pr[i][e] = __shfl_xor_sync(0xffffffffu, x[i][e], h16);
-    } else {
-      // rotated slice of 512 dims: the partner chunk is this lane's other chunk
-#pragma unroll
-      for (int i = 0; i < NCH; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pr[i][e] = x[NCH - 1 - i][e];
-    }
-    const float2* trow = la.rope_tab + static_cast<size_t>(pos) * half;
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int c = lane + 32 * i;
-      if (8 * c < la.rot) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int d = 8 * c + e;
-          const bool first = d < half;
-          const float2 cs = __ldg(trow + (first ? d : d - half));
-          x[i][e] = first ? x[i][e] * cs.x - pr[i][e] * cs.y : x[i][e] * cs.x + pr[i][e] * cs.y;
-        }
-      }
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------

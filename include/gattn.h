@@ -93,9 +93,7 @@ typedef struct {
 /* ---- RoPE table ---------------------------------------------------------
  * Table of (cos, sin) pairs, fp32, layout [max_pos][rot_dim/2][2], with
  * angle(p, t) = p * theta^(-2t/freq_dim) evaluated in double precision and
- * rounded once to fp32, followed by rot_dim/2 doubles theta^(-2t/freq_dim)/(2 pi)
- * (the angle of one position step in turns, used where a kernel computes the
- * angle itself).  Build it once per (theta, rot_dim, freq_dim) and
+ * rounded once to fp32.  Build it once per (theta, rot_dim, freq_dim) and
  * pass it in gattn_cfg.rope_table.
  * gattn_rope_table_bytes returns 0 for invalid sizes.
  * gattn_rope_table_fill returns INVALID_ARG for a NULL/misaligned table,
