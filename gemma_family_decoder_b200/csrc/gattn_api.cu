@@ -6,7 +6,6 @@
 
 #include <cmath>
 #include <cstdio>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -285,9 +284,7 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   pa.trace = static_cast<unsigned long long*>(g_trace_buf);
   pa.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
-  static const bool pair_off = getenv("GATTN_NO_PAIR") != nullptr;  // temporary A/B knob
-  cudaError_t e = (!pair_off && gattn::prefill_pair_supported(la)) ? gattn::launch_prefill_pair(pa, la, s)
-                                                                  : gattn::launch_prefill(pa, la, s);
+  cudaError_t e = gattn::launch_prefill(pa, la, s);
   if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
   if (e != cudaSuccess) return fail_cuda(e, "prefill launch");
   return GATTN_OK;

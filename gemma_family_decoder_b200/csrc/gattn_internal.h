@@ -68,9 +68,6 @@ struct PrefillArgs {
   size_t trace_bytes;
 };
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
-// Head_dim 256 with an even query-group size: pairs of SMs share each K/V tile.
-bool prefill_pair_supported(const LayerArgs& la);
-cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
 
 // Self-test: one CTA waits on an mbarrier nobody arrives on.
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t s);

@@ -33,11 +33,7 @@ namespace gattn {
 
 using bf16 = __nv_bfloat16;
 
-// QTM: the transformed Q tile lives in tensor memory (A operand of Q K^T read
-// from TMEM) instead of shared memory.  It needs Q (D/2 columns), O (256), and
-// two S slots to fit the 512 TMEM columns, so it is used at head_dim 256 with
-// 64-key tiles; the raw Q tile is staged through the first ring slots.
-template <int D, int BN, bool QTM>
+template <int D, int BN>
 struct PrefillShape {
   static constexpr int BM = 128;
   static constexpr int DV = 256;                 // value dims per CTA
@@ -45,12 +41,11 @@ struct PrefillShape {
   static constexpr int KCH = D / 64;             // slots per key tile
   static constexpr int VCH = DV / 64;            // slots per value tile
   static constexpr int SLAB128 = BM * 128;       // 64 dims x 128 rows
-  static constexpr int Q_BYTES = QTM ? 0 : (D / 64) * SLAB128;
-  static constexpr int QSLOTS = QTM ? (D / 64) * SLAB128 / SLAB_KV : 0;  // ring slots staging Q
+  static constexpr int Q_BYTES = (D / 64) * SLAB128;
   // ring slots: a multiple of 4 so that every 4-slot value tile is contiguous
   static constexpr int NSTAGE = ((227 * 1024 - Q_BYTES - 2048) / SLAB_KV) / 4 * 4;
   static constexpr int OFF_RING = Q_BYTES;
-  static constexpr int OFF_Q = QTM ? OFF_RING : 0;  // raw Q tile (and later the O tile)
+  static constexpr int OFF_Q = 0;  // Q tile (and later the O tile)
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * SLAB_KV;
   static constexpr int NBAR = 2 * NSTAGE + 10;
   static_assert(NSTAGE >= KCH + VCH, "ring must hold a key tile and a value tile");
@@ -58,15 +53,12 @@ struct PrefillShape {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr uint32_t TM_O = 0;
-  static constexpr uint32_t TM_Q = DV;                       // QTM only: D/2 columns
-  static constexpr uint32_t TM_S0 = QTM ? DV + D / 2 : DV;
+  static constexpr uint32_t TM_S0 = DV;
   static constexpr uint32_t TM_S1 = TM_S0 + BN;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(TM_S1 + BN <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert((QTM ? NSTAGE * SLAB_KV : Q_BYTES) >= BM * DV * 2,
-                "the output tile reuses the Q staging area");
-  static_assert(!QTM || (QSLOTS <= NSTAGE && QSLOTS % 4 == 0), "Q staging slots");
+  static_assert(Q_BYTES >= BM * DV * 2, "the output tile reuses the Q tile's shared memory");
 };
 
 struct PrefillKParams {
@@ -92,9 +84,9 @@ constexpr int kTraceSlots = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, int BN, bool CAP, bool QTM>
+template <int D, int BN, bool CAP>
 __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ PrefillKParams P) {
-  using C = PrefillShape<D, BN, QTM>;
+  using C = PrefillShape<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
@@ -188,16 +180,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     const int qi = q0 + t;
     const bool valid = qi < S;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    bool ok;
-    if constexpr (QTM) {
-      bool got = true;
-      for (int sl = 0; sl < C::QSLOTS; ++sl) got = got && mbar_wait(&full[sl], 0, tmo, P.status, abort_flag);
-      ok = __all_sync(0xffffffffu, got);
-    } else {
-      ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
-    }
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
 
-    // query prologue in place: RMSNorm + RoPE in fp32 on this thread's row
     // query prologue in place, thread t on row t; RoPE angles computed, not read
     if (ok && valid && (la.rot > 0 || la.qk_norm)) {
       int pos = la.rot > 0 ? __ldg(P.positions + static_cast<size_t>(b) * S + qi) : 0;
@@ -210,28 +194,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
                                   : 1.f;
       tile_row_prologue(smem + C::OFF_Q, C::SLAB128, t, pos, la, rn, 0, la.rot >> 4, la.rot >> 3, D / 8);
     }
-    if constexpr (QTM) {
-      // move this thread's row into the Q columns of TMEM (64 dims per x32 store)
-      const uint8_t* qrow = smem + C::OFF_Q + t * 128;
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t v[32];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 u = *reinterpret_cast<const uint4*>(qrow + cc * C::SLAB128 + ((k ^ (t & 7)) << 4));
-          v[4 * k] = u.x; v[4 * k + 1] = u.y; v[4 * k + 2] = u.z; v[4 * k + 3] = u.w;
-        }
-        tmem_st32(tmem + lane_off + C::TM_Q + cc * 32, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      named_barrier(1, 128);
-      // the staging slots go back to the producer as consumed ring slots
-      if (t == 0)
-        for (int sl = 0; sl < C::QSLOTS; ++sl) mbar_arrive(&empty[sl]);
-    } else {
-      fence_proxy_async_smem();
-    }
+    fence_proxy_async_smem();
     mbar_arrive(q_ready);
 
     // main loop over KV tiles
@@ -362,21 +325,10 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       int n = 0;
-      if constexpr (QTM) {
-        // raw Q tile through the first ring slots: slot 2c + r holds rows
-        // [64r, 64r+64) of dims [64c, 64c+64), i.e. one 128-row slab per 2 slots
-        for (int sl = 0; sl < C::QSLOTS; ++sl) {
-          mbar_arrive_expect_tx(&full[sl], C::SLAB_KV);
-          tma_load_4d(smem + C::OFF_RING + sl * C::SLAB_KV, &P.tm_q, &full[sl], (sl >> 1) * 64, h,
-                      q0 + (sl & 1) * 64, b);
-        }
-        n = C::QSLOTS;
-      } else {
-        mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
-        for (int sl = 0; sl < D / 64; ++sl)
-          tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
-      }
+      for (int sl = 0; sl < D / 64; ++sl)
+        tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
       auto load = [&](const CUtensorMap* tm, int d0, int key0) -> bool {
         const int st = n % C::NSTAGE;
         const uint32_t par = ((n / C::NSTAGE) & 1) ^ 1;
@@ -395,7 +347,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       }
       for (int c = 0; c < C::VCH && ok; ++c) ok = load(&P.tm_v, dv_lo + c * 64, tile_key(ntiles - 1));
       // let every issued copy land before the CTA can exit
-      if constexpr (!QTM) mbar_wait(q_full, 0, tmo, P.status, nullptr);
+      mbar_wait(q_full, 0, tmo, P.status, nullptr);
       for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)
         mbar_wait(&full[i % C::NSTAGE], (i / C::NSTAGE) & 1, tmo, P.status, nullptr);
     }
@@ -404,7 +356,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
-      int n = C::QSLOTS;
+      int n = 0;
       bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
       mark(3);
       tc_fence_after();
@@ -420,12 +372,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bd = smem_desc_sw128(kb + kk * 32, 16, 1024);
-            if constexpr (QTM) {
-              mma_bf16_ts(s_tm, tmem + C::TM_Q + c * 32 + kk * 8, bd, idesc_qk, (c | kk) != 0);
-            } else {
-              const uint64_t a = smem_desc_sw128(qb + kk * 32, 16, 1024);
-              mma_bf16_ss(s_tm, a, bd, idesc_qk, (c | kk) != 0);
-            }
+            const uint64_t a = smem_desc_sw128(qb + kk * 32, 16, 1024);
+            mma_bf16_ss(s_tm, a, bd, idesc_qk, (c | kk) != 0);
           }
           mma_commit(&empty[st]);
           ++n;
@@ -481,11 +429,11 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   if (threadIdx.x == 0) mark(5);
 }
 
-template <int D, int BN, bool CAP, bool QTM>
+template <int D, int BN, bool CAP>
 static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
-  using C = PrefillShape<D, BN, QTM>;
+  using C = PrefillShape<D, BN>;
   PrefillKParams P;
-  if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, D, QTM ? 64 : C::BM) ||
+  if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, D, C::BM) ||
       !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN) ||
       !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN) ||
       !encode_tmap_bshd(&P.tm_o, pa.out, pa.B, pa.S, la.H, D, C::BM))
@@ -500,7 +448,7 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.la = la;
   P.trace = pa.trace;
   P.trace_ctas = static_cast<int>(pa.trace_bytes / (kTraceSlots * sizeof(unsigned long long)));
-  auto kern = prefill_kernel<D, BN, CAP, QTM>;
+  auto kern = prefill_kernel<D, BN, CAP>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -515,9 +463,9 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   const bool cap = la.softcap > 0.f;
   if (la.D == 256)
-    return cap ? run_prefill<256, 64, true, true>(pa, la, s) : run_prefill<256, 64, false, true>(pa, la, s);
+    return cap ? run_prefill<256, 128, true>(pa, la, s) : run_prefill<256, 128, false>(pa, la, s);
   if (la.D == 512)
-    return cap ? run_prefill<512, 64, true, false>(pa, la, s) : run_prefill<512, 64, false, false>(pa, la, s);
+    return cap ? run_prefill<512, 64, true>(pa, la, s) : run_prefill<512, 64, false>(pa, la, s);
   return cudaErrorInvalidValue;
 }
 
