@@ -53,6 +53,10 @@ struct DecodeArgs {
 void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk);
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
+// Tensor-core split kernel: K=V layers with 8 or 16 query heads per kv head,
+// head_dim 256 or 512 and at most 128 rotated dims (same partial format).
+bool decode_tc_supported(const DecodeArgs& da, const LayerArgs& la);
+cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 
 // Prefill on tcgen05 tensor cores.
 struct PrefillArgs {

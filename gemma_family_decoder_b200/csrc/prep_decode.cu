@@ -291,6 +291,7 @@ static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, c
 }
 
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  if (decode_tc_supported(da, la)) return launch_decode_tc(da, la, s);
   const int hpw = la.G <= 2 ? la.G : la.G / 4;
   if (la.D == 256) {
     switch (hpw) {

@@ -180,6 +180,17 @@ DEC_CASES = [
     ("mqa_d256_softcap_norm1", W.Layer(num_heads=8, num_kv_heads=1, head_dim=256, softcap=50.0,
                                        qk_norm=W.NORM_ONE_PLUS_W, window=300), [1, 299, 300, 301, 900]),
     ("gqa4_d256", W.Layer(num_heads=16, num_kv_heads=4, head_dim=256, rope_theta=1e6), [7, 600]),
+    # tensor-core split kernel (K=V, 8 or 16 query heads per kv head, <= 128 rotated dims)
+    ("keqv_g8_d512_norm", W.Layer(num_heads=8, num_kv_heads=1, head_dim=512, rope_theta=1e6,
+                                  rotary_fraction=0.25, scalar=512.0, k_eq_v=True,
+                                  qk_norm=W.NORM_W), [3, 64, 65, 700]),
+    ("keqv_g16_d256_cap_r16", W.Layer(num_heads=32, num_kv_heads=2, head_dim=256,
+                                      rotary_fraction=0.0625, softcap=30.0, k_eq_v=True,
+                                      qk_norm=W.NORM_ONE_PLUS_W, window=200),
+     [1, 150, 199, 200, 201, 1300]),
+    ("keqv_g16_d512_w512", W.Layer(num_heads=16, num_kv_heads=1, head_dim=512, window=512,
+                                   rotary_fraction=0.25, scalar=512.0, k_eq_v=True),
+     [100, 513, 2000]),
 ]
 
 
