@@ -41,10 +41,10 @@ struct DecShape {
   static constexpr int OFF_ROT = OFF_RAW + NSTAGE * RAW;
   static constexpr int OFF_Q = OFF_ROT + NSTAGE * ROTB * BOX;
   static constexpr int OFF_P = OFF_Q + NB * QSLAB;
-  static constexpr int OFF_RN = OFF_P + NSTAGE * PSLAB;     // 1/rms(k) per key, [2][64]
-  static constexpr int OFF_RED = OFF_RN + NSTAGE * TK * 4;  // head maxima [2][4][G], sums [4][G]
+  static constexpr int OFF_RSTEP = OFF_P + NSTAGE * PSLAB;  // (cos, sin) of a 64-position step, [64]
+  static constexpr int OFF_RED = OFF_RSTEP + 64 * 8;        // head maxima [2][4][G], sums [4][G]
   static constexpr int OFF_BAR = OFF_RED + 3 * 4 * G * 4;
-  static constexpr int NBAR = 18;
+  static constexpr int NBAR = 16;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TM_S0 = 0;           // S^T slots: G columns each
@@ -95,19 +95,17 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;            // [2] raw tile landed (TMA bytes)
-  uint64_t* raw_empty = bars + 2;   // [2] P V done with the raw tile
+  uint64_t* raw_empty = bars + 2;   // [2] P V done with the raw tile and P^T slot
   uint64_t* rot_full = bars + 4;    // [2] key prologue done (128 arrivals)
   uint64_t* rot_empty = bars + 6;   // [2] Q K^T done with the side tile
   uint64_t* s_full = bars + 8;      // [2] S^T ready
-  uint64_t* p_full = bars + 10;     // [2] P^T written, O rescaled (128 arrivals)
-  uint64_t* rn_empty = bars + 12;   // [2] softmax has read the tile's key norms (128 arrivals)
-  uint64_t* o_done = bars + 14;     // one phase per P V
-  uint64_t* o_final = bars + 15;
-  uint64_t* q_ready = bars + 16;    // 128 arrivals
-  uint64_t* drain = bars + 17;
+  uint64_t* p_full = bars + 10;     // [2] P^T written, O rescaled, S read (128 arrivals)
+  // bars + 12: unused
+  uint64_t* o_final = bars + 13;
+  uint64_t* q_ready = bars + 14;    // 256 arrivals (warps 0-7)
+  uint64_t* drain = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  float* rnorm = reinterpret_cast<float*>(smem + C::OFF_RN);   // [2][64]
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);    // [3][4][G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,11 +117,9 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       mbar_init(&rot_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
-      mbar_init(&rn_empty[i], 128);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -138,56 +134,82 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = P.timeout_ns;
-  if (warp < 4) {
-    // ------------------------------------------- query prologue, softmax, epilogue
+  // optional timeline of this CTA (512 entries; layout in the public header)
+  const long long cta = (static_cast<long long>(b) * la.Hkv + kvh) * da.nsplit + split;
+  unsigned long long* trace =
+      (da.trace && cta < static_cast<long long>(da.trace_bytes / (512 * sizeof(unsigned long long))))
+          ? da.trace + cta * 512 : nullptr;
+  const uint64_t t_start = trace ? globaltimer_ns() : 0;
+  auto mark = [&](int slot) {
+    if (trace) trace[slot] = globaltimer_ns() - t_start;
+  };
+  if (trace && threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    trace[0] = t_start;
+    trace[1] = smid;
+    trace[2] = ntiles;
+  }
+  if (warp < 8) {
+    // ------------------------------------------------------------ query rows
+    // Warps 0-7, one head per warp at a time: QK-norm and RoPE at position L-1
+    // into the Q^T operand.  On the unrotated dims the key's gain is applied
+    // here instead of to the keys.  Every row is loaded before any is
+    // transformed, so the global reads overlap.
     constexpr int NCH = D / 256;
+    constexpr int HPW = (G + 7) / 8;
+    const float koff = la.qk_norm == 1 ? 1.f : 0.f;
+    const float4* gk4 = reinterpret_cast<const float4*>(la.k_norm_w);
+    float x[HPW][NCH][8];
+#pragma unroll
+    for (int hh = 0; hh < HPW; ++hh) load_row<NCH>(da.q + (head0 + warp + 8 * hh) * D, lane, x[hh]);
+#pragma unroll
+    for (int hh = 0; hh < HPW; ++hh) {
+      const int h = warp + 8 * hh;
+      transform_row<NCH>(x[hh], lane, L - 1, la, la.q_norm_w, da.status);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int c = lane + 32 * i;  // 8-dim chunk
+        if (la.qk_norm && 8 * c >= la.rot) {
+          const float4 g0 = __ldg(gk4 + 2 * c), g1 = __ldg(gk4 + 2 * c + 1);
+          x[hh][i][0] *= g0.x + koff; x[hh][i][1] *= g0.y + koff;
+          x[hh][i][2] *= g0.z + koff; x[hh][i][3] *= g0.w + koff;
+          x[hh][i][4] *= g1.x + koff; x[hh][i][5] *= g1.y + koff;
+          x[hh][i][6] *= g1.z + koff; x[hh][i][7] *= g1.w + koff;
+        }
+        *reinterpret_cast<uint4*>(smem + C::OFF_Q + (c >> 3) * C::QSLAB + h * 128 +
+                                  (((c & 7) ^ (h & 7)) << 4)) = pack8(x[hh][i]);
+      }
+    }
+    // P^T rows past the group (N padding of P V) stay zero
+    if constexpr (C::NPV > G) {
+      for (int i = threadIdx.x; i < 2 * (C::NPV - G) * 8; i += 256) {
+        const int sl = i / ((C::NPV - G) * 8), r = i % ((C::NPV - G) * 8);
+        *reinterpret_cast<uint4*>(smem + C::OFF_P + sl * C::PSLAB + G * 128 + r * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+  }
+  if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    // Thread (warp w, lane i) serves key kt = 16 w + i%16 of each tile: lanes
+    // i and i+16 sum the squares of its two halves of dims (the key's norm,
+    // taken while the rotation and Q K^T run), and lane i < 16 reads its row
+    // of S^T (TMEM lane 32 w + i holds row 16 w + i of an M=64 accumulator)
+    // with the logits of all G heads.  Maxima are per head over the 64 keys
+    // (warp shuffles, then the 4 warps through shared memory); the running
+    // max m is the same in every thread, so the rescale decision is uniform
+    // over the warpgroup.
     const int t = threadIdx.x;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    // Query rows: QK-norm and RoPE at position L-1, one warp per head.  On the
-    // unrotated dims the key's gain is applied here instead of to the keys.
-    {
-      const float koff = la.qk_norm == 1 ? 1.f : 0.f;
-      const float4* gk4 = reinterpret_cast<const float4*>(la.k_norm_w);
-      for (int h = warp; h < G; h += 4) {
-        float x[NCH][8];
-        load_row<NCH>(da.q + (head0 + h) * D, lane, x);
-        transform_row<NCH>(x, lane, L - 1, la, la.q_norm_w, da.status);
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-          const int c = lane + 32 * i;  // 8-dim chunk
-          if (la.qk_norm && 8 * c >= la.rot) {
-            const float4 g0 = __ldg(gk4 + 2 * c), g1 = __ldg(gk4 + 2 * c + 1);
-            x[i][0] *= g0.x + koff; x[i][1] *= g0.y + koff;
-            x[i][2] *= g0.z + koff; x[i][3] *= g0.w + koff;
-            x[i][4] *= g1.x + koff; x[i][5] *= g1.y + koff;
-            x[i][6] *= g1.z + koff; x[i][7] *= g1.w + koff;
-          }
-          *reinterpret_cast<uint4*>(smem + C::OFF_Q + (c >> 3) * C::QSLAB + h * 128 +
-                                    (((c & 7) ^ (h & 7)) << 4)) = pack8(x[i]);
-        }
-      }
-      // P^T rows past the group (N padding of P V) stay zero
-      if constexpr (C::NPV > G) {
-        for (int i = t; i < 2 * (C::NPV - G) * 8; i += 128) {
-          const int sl = i / ((C::NPV - G) * 8), r = i % ((C::NPV - G) * 8);
-          *reinterpret_cast<uint4*>(smem + C::OFF_P + sl * C::PSLAB + G * 128 + r * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(q_ready);
-    }
-
-    // Softmax over each tile's S^T: thread (warp w, lane i < 16) owns key
-    // 16 w + i, TMEM lane 32 w + i, and the logits of all G heads in its row.
-    // Maxima are per head over the 64 keys (warp shuffles, then the 4 warps
-    // through shared memory); the running max m is the same in every thread,
-    // so the rescale decision is uniform over the warpgroup.
     const bool cap = la.softcap > 0.f;
     const float sl2 = la.scale_log2;
     const float kcap = cap ? la.scale / la.softcap : 0.f;
     const float cap_l2 = cap ? la.softcap * kLog2eD : 0.f;
     const int kt = 16 * warp + (lane & 15);  // key within the tile
+    const int half = lane >> 4;
     const bool key_lane = lane < 16;
     float m[G], lp[G];
 #pragma unroll
@@ -199,16 +221,35 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     for (int j = 0; j < ntiles; ++j) {
       const int slot = j & 1;
       const uint32_t par = (j >> 1) & 1;
-      const bool okj =
-          ok && __all_sync(0xffffffffu, mbar_wait(&s_full[slot], par, tmo, da.status, abort_flag) &&
-                                            mbar_wait(&rot_full[slot], par, tmo, da.status, abort_flag));
+      bool okj = ok && __all_sync(0xffffffffu, mbar_wait(&full[slot], par, tmo, da.status, abort_flag));
+      float rn = 1.f;
+      if (la.qk_norm) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        if (okj) {
+          uint8_t* raw = smem + C::OFF_RAW + slot * C::RAW;
+#pragma unroll 4
+          for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c) {
+            float xx[8];
+            unpack8(*tile_chunk(raw, C::BOX, kt, c), xx);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(xx[e], xx[e], acc[e]);
+          }
+        }
+        float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+        rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
+      }
+      if (t == 0 && j < 24) mark(176 + j);
+      okj = okj && __all_sync(0xffffffffu, mbar_wait(&s_full[slot], par, tmo, da.status, abort_flag));
+      if (t == 0 && j < 24) mark(80 + j);
       float x[G];
       if (okj) {
         tc_fence_after();
         uint32_t sr[G];
         tmem_ldg<G>(tmem + lane_off + (slot ? C::TM_S1 : C::TM_S0), sr);
         tmem_wait_ld();
-        const float rn = rnorm[slot * C::TK + kt];
         const bool vis = key_lane && (start + j * C::TK + kt) < end;
         const float f = rn * (cap ? kcap : sl2);
 #pragma unroll
@@ -220,50 +261,76 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
 #pragma unroll
         for (int h = 0; h < G; ++h) x[h] = -INFINITY;
       }
-      mbar_arrive(&rn_empty[slot]);
-      float* rw = red + (slot * 4 + warp) * G;
+      // The running max moves only when a logit passes it by more than 8
+      // (log2 units, a factor 256): the warpgroup votes, and exchanges the
+      // tile's maxima only then.  Every thread of the warpgroup leaves the
+      // loop at the exchange or not at all.
+      bool need = !okj;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = x[h];
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-        if (lane == 0) rw[h] = v;
-      }
-      // every thread of the warpgroup leaves the loop at this barrier or not at all
-      ok = named_barrier_and(1, 128, okj);
-      if (!ok) break;
-      const float* rr = red + slot * 4 * G;
+      for (int h = 0; h < G; ++h) need = need || x[h] > m[h] + 8.f;
       float alpha[G];
-      bool any = false;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float mt = fmaxf(fmaxf(rr[h], rr[G + h]), fmaxf(rr[2 * G + h], rr[3 * G + h]));
-        const float mn = fmaxf(m[h], mt);
-        alpha[h] = 1.f;
-        if (mn > m[h] + 8.f) {  // lazy rescale: the reference max moves only by > 2^8
-          alpha[h] = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
-          any = any || m[h] != -INFINITY;
-          m[h] = mn;
+      for (int h = 0; h < G; ++h) alpha[h] = 1.f;
+      bool any = false;
+      if (named_barrier_or(1, 128, need)) {
+        float* rw = red + (slot * 4 + warp) * G;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float v = x[h];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          if (lane == 0) rw[h] = v;
+        }
+        ok = named_barrier_and(1, 128, okj);
+        if (!ok) break;
+        const float* rr = red + slot * 4 * G;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float mt = fmaxf(fmaxf(rr[h], rr[G + h]), fmaxf(rr[2 * G + h], rr[3 * G + h]));
+          const float mn = fmaxf(m[h], mt);
+          if (mn > m[h] + 8.f) {
+            alpha[h] = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
+            any = any || m[h] != -INFINITY;
+            m[h] = mn;
+          }
         }
       }
-      // P^T row h is one 128-byte swizzled row: key k at chunk (k/8) ^ (h%8), half-word k%8
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float mu = m[h] == -INFINITY ? 0.f : m[h];
-        const float p = ex2(x[h] - mu);
-        lp[h] = lp[h] * alpha[h] + p;
-        if (key_lane)
-          *reinterpret_cast<__nv_bfloat16*>(smem + C::OFF_P + slot * C::PSLAB + h * 128 +
-                                            (((kt >> 3) ^ (h & 7)) << 4) + (kt & 7) * 2) =
-              __float2bfloat16_rn(p);
+      if (t == 0 && j < 24) mark(200 + j);
+      // P^T slot reuse: P V(j-2), which read it, must be complete
+      if (j >= 2) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&raw_empty[slot], par ^ 1, tmo, da.status, abort_flag)))
+          ok = false;
       }
-      // O must hold P V of every earlier tile before it is rescaled.  Seeing
-      // S(j) implies P V(j-2) is complete (it was issued before Q K^T(j)), so
-      // o_done is at most one phase behind and the parity wait is exact.
+      if (t == 0 && j < 24) mark(248 + j);
+      // P^T row h is one 128-byte swizzled row: key k at chunk (k/8) ^ (h%8),
+      // half-word k%8.  Lanes 2i and 2i+1 (adjacent keys) swap one value so
+      // that each writes a 32-bit word: the even lane for even heads, the odd
+      // lane for odd heads.
+      {
+        uint8_t* pbase = smem + C::OFF_P + slot * C::PSLAB;
+        const int kp = kt & ~1;
+        const bool odd = lane & 1;
+#pragma unroll
+        for (int h = 0; h < G; h += 2) {
+          const float p0 = ex2(x[h] - (m[h] == -INFINITY ? 0.f : m[h]));
+          const float p1 = ex2(x[h + 1] - (m[h + 1] == -INFINITY ? 0.f : m[h + 1]));
+          lp[h] = lp[h] * alpha[h] + p0;
+          lp[h + 1] = lp[h + 1] * alpha[h + 1] + p1;
+          const float recv = __shfl_xor_sync(0xffffffffu, odd ? p0 : p1, 1);
+          if (key_lane) {
+            const int hh = h + (odd ? 1 : 0);
+            *reinterpret_cast<uint32_t*>(pbase + hh * 128 + (((kp >> 3) ^ (hh & 7)) << 4) + (kp & 7) * 2) =
+                odd ? pack_bf16x2(recv, p1) : pack_bf16x2(p0, recv);
+          }
+        }
+      }
+      if (t == 0 && j < 24) mark(224 + j);
+      // O must hold P V of every earlier tile before it is rescaled
       if (any && j >= 1) {
-        const bool okw = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, da.status, abort_flag));
+        const bool okw = __all_sync(0xffffffffu, mbar_wait(&raw_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, tmo,
+                                                           da.status, abort_flag));
         if (okw) {
           tc_fence_after();
 #pragma unroll
@@ -283,8 +350,8 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[slot]);
+      if (lane == 0 && j < 24) mark((t == 0 ? 104 : 368 + 24 * warp) + j);
     }
-
     // Epilogue: l summed over the tile's keys and the 4 warps; thread t writes
     // value dim 128 c + t of each head's unnormalised O, lane t < G the (m, l)
     // of head t, in the split kernel's partial format.
@@ -301,6 +368,7 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     }
     ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, tmo, da.status, abort_flag));
     ok = named_barrier_and(1, 128, ok);
+    if (t == 0) mark(4);
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
@@ -324,25 +392,46 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   }
   else if (warp < 8) {
     // ------------------------------------------------------------ key prologue
-    // Two threads per key (t4 = 2 k + hf).  Per tile: 1/rms of the raw key row
-    // into rnorm, the rotated dims [0, R) of k * gain into the side tile with
-    // angles computed here (pair t turns theta^(-2t/F) / 2pi per position, a
-    // geometric sequence in double precision), and zero rows for keys past
-    // the chunk's end, so that P V multiplies 0 by 0 there, not by stale data.
+    // Two threads per key (t4 = 2 k + hf) write the rotated dims [0, R) of
+    // k * gain into the side tile, and zero rows for keys past the chunk's end
+    // so that P V multiplies 0 by 0 there, not by stale data.  Each thread
+    // keeps (cos, sin) of its pairs' angles at its key's position: computed
+    // exactly (pair t turns theta^(-2t/F) / 2pi per position, a geometric
+    // sequence in double precision, reduced mod 1) every 32 tiles, and in
+    // between advanced by the 64-position step of each pair.
     const int t4 = threadIdx.x - 128;
     const int k = t4 >> 1, hf = t4 & 1;
     const int R = la.rot;
-    const int h8 = R >> 4;                  // 8-dim chunks in half the rotated slice
+    const int h8 = R >> 4;                  // 8-dim chunks in half the rotated slice (<= 8)
     const int rch = ((R + 63) >> 6) << 3;   // chunks covered by the side tile's boxes
     const float koff = la.qk_norm == 1 ? 1.f : 0.f;
     const float4* gk4 = reinterpret_cast<const float4*>(la.k_norm_w);
-    double qp[8];
-    qp[0] = 1.0;
+    float2* rstep = reinterpret_cast<float2*>(smem + C::OFF_RSTEP);
+    constexpr double kTurnsPerRad = 0.15915494309189533576888376337251;
+    if (t4 < (R >> 1)) {
+      double f = kTurnsPerRad;
+      for (int i = 0; i < t4; ++i) f *= la.rope_ratio;
+      rstep[t4] = rope_cos_sin(C::TK, f);
+    }
+    named_barrier(2, 128);
+    float2 cs[4][8];
+    auto anchor = [&](int pos) {
+      double qp[8];
+      qp[0] = 1.0;
 #pragma unroll
-    for (int e = 1; e < 8; ++e) qp[e] = qp[e - 1] * la.rope_ratio;
-    const double q8 = qp[7] * la.rope_ratio;
-    const double q16 = q8 * q8;
-    const double f_first = 0.15915494309189533576888376337251 * (hf ? q8 : 1.0);
+      for (int e = 1; e < 8; ++e) qp[e] = qp[e - 1] * la.rope_ratio;
+      const double q8 = qp[7] * la.rope_ratio;
+      const double q16 = q8 * q8;
+      double f8 = kTurnsPerRad * (hf ? q8 : 1.0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (hf + 2 * i < h8) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) cs[i][e] = rope_cos_sin(pos, f8 * qp[e]);
+        }
+        f8 *= q16;
+      }
+    };
     auto gain8 = [&](int c, float (&x)[8]) {
       if (!la.qk_norm) return;
       const float4 g0 = __ldg(gk4 + 2 * c), g1 = __ldg(gk4 + 2 * c + 1);
@@ -352,116 +441,92 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     for (int j = 0; j < ntiles; ++j) {
       const int slot = j & 1;
       const uint32_t par = (j >> 1) & 1;
-      // warp-uniform exit: the norm's pair shuffle below needs every lane
       if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], par, tmo, da.status, abort_flag) &&
-                                       mbar_wait(&rot_empty[slot], par ^ 1, tmo, da.status, abort_flag) &&
-                                       mbar_wait(&rn_empty[slot], par ^ 1, tmo, da.status, abort_flag)))
+                                       mbar_wait(&rot_empty[slot], par ^ 1, tmo, da.status, abort_flag)))
         break;
+      if (t4 == 0 && j < 24) mark(8 + j);
       uint8_t* raw = smem + C::OFF_RAW + slot * C::RAW;
       uint8_t* rot = smem + C::OFF_ROT + slot * C::ROTB * C::BOX;
       const int key = start + j * C::TK + k;
-      float rn = 1.f;
-      if (la.qk_norm) {
-        float ss = 0.f;
-#pragma unroll 4
-        for (int c = hf; c < D / 8; c += 2) {
-          float x[8];
-          unpack8(*tile_chunk(raw, C::BOX, k, c), x);
+      if (R > 0) {
+        if ((j & 31) == 0) {
+          anchor(checked_pos(min(key, end - 1), la, da.status));
+        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-        }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
-      }
-      if (key < end) {
-        if (hf == 0) rnorm[slot * C::TK + k] = rn;
-        if (R > 0) {
-          const int pos = checked_pos(key, la, da.status);
-          double f8 = f_first;
-          for (int c = hf; c < h8; c += 2) {
-            float x[8], y[8];
-            unpack8(*tile_chunk(raw, C::BOX, k, c), x);
-            unpack8(*tile_chunk(raw, C::BOX, k, c + h8), y);
-            gain8(c, x);
-            gain8(c + h8, y);
-            float xo[8], yo[8];
+          for (int i = 0; i < 4; ++i) {
+            const int c = hf + 2 * i;
+            if (c < h8) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float2 cs = rope_cos_sin(pos, f8 * qp[e]);
-              xo[e] = x[e] * cs.x - y[e] * cs.y;
-              yo[e] = y[e] * cs.x + x[e] * cs.y;
+              for (int e = 0; e < 8; ++e) {
+                const float2 st = rstep[8 * c + e];
+                const float2 a = cs[i][e];
+                cs[i][e] = make_float2(a.x * st.x - a.y * st.y, a.y * st.x + a.x * st.y);
+              }
             }
-            *tile_chunk(rot, C::BOX, k, c) = pack8(xo);
-            *tile_chunk(rot, C::BOX, k, c + h8) = pack8(yo);
-            f8 *= q16;
+          }
+        }
+      }
+      if (t4 == 0 && j < 24) mark(296 + j);
+      if (key < end) {
+        if (R > 0) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = hf + 2 * i;
+            if (c < h8) {
+              float x[8], y[8];
+              unpack8(*tile_chunk(raw, C::BOX, k, c), x);
+              unpack8(*tile_chunk(raw, C::BOX, k, c + h8), y);
+              gain8(c, x);
+              gain8(c + h8, y);
+              float xo[8], yo[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                xo[e] = x[e] * cs[i][e].x - y[e] * cs[i][e].y;
+                yo[e] = y[e] * cs[i][e].x + x[e] * cs[i][e].y;
+              }
+              *tile_chunk(rot, C::BOX, k, c) = pack8(xo);
+              *tile_chunk(rot, C::BOX, k, c + h8) = pack8(yo);
+            }
           }
           // unrotated dims that share a box with rotated ones: copied raw
           for (int c = 2 * h8 + hf; c < rch; c += 2) *tile_chunk(rot, C::BOX, k, c) = *tile_chunk(raw, C::BOX, k, c);
         }
       } else {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        if (hf == 0) rnorm[slot * C::TK + k] = 0.f;
         for (int c = hf; c < D / 8; c += 2) *tile_chunk(raw, C::BOX, k, c) = z;
         for (int c = hf; c < rch; c += 2) *tile_chunk(rot, C::BOX, k, c) = z;
       }
       fence_proxy_async_smem();
       mbar_arrive(&rot_full[slot]);
+      if ((t4 & 31) == 0 && j < 24) mark((t4 == 0 ? 32 : 296 + t4 * 3 / 4) + j);
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+  }
+  else if (warp == 8) {
+    // ------------------------------------------------- TMA producer, P V issuer
+    // One thread loads tiles 0 and 1, then per tile j issues
+    // O^T += V^T P^T once the softmax has written P^T(j): A = value boxes
+    // (MN-major, M=128 dims over two 64-dim boxes LBO apart), B = P^T
+    // (K-major, N=NPV); and once that P V has completed, loads tile j+2 into
+    // the slot it frees.
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < ntiles; ++j) {
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NPV, true, false);
+      auto load = [&](int j) {
         const int slot = j & 1;
-        if (!mbar_wait(&raw_empty[slot], ((j >> 1) & 1) ^ 1, tmo, da.status, abort_flag)) break;
         mbar_arrive_expect_tx(&full[slot], C::RAW);
 #pragma unroll
         for (int c = 0; c < C::NB; ++c)
           tma_load_4d(smem + C::OFF_RAW + slot * C::RAW + c * C::BOX, &P.tm_k, &full[slot], 64 * c,
                       kvh, start + j * C::TK, b);
-        issued = j + 1;
-      }
-      // let every issued copy land before the CTA can exit
-      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-        mbar_wait(&full[j & 1], (j >> 1) & 1, tmo, da.status, nullptr);
-    }
-  } else {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      // S^T = K~ Q~^T: A = key box (K-major, M=64), B = Q^T slab (K-major, N=G).
-      // O^T += V^T P^T: A = value boxes (MN-major, M=128 dims over two 64-dim
-      // boxes LBO apart), B = P^T (K-major, N=NPV).
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(64, G, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NPV, true, false);
-      const int rotb = (la.rot + 63) >> 6;
-      bool ok = mbar_wait(q_ready, 0, tmo, da.status, abort_flag);
-      tc_fence_after();
-      auto qk = [&](int j) -> bool {
+        if (j < 24) mark(152 + j);
+      };
+      int issued = 0;
+      for (; issued < 2 && issued < ntiles; ++issued) load(issued);
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j) {
         const int slot = j & 1;
         const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(&full[slot], par, tmo, da.status, abort_flag) ||
-            !mbar_wait(&rot_full[slot], par, tmo, da.status, abort_flag))
-          return false;
-        tc_fence_after();
-        const uint32_t s_tm = tmem + (slot ? C::TM_S1 : C::TM_S0);
-        const uint32_t rawb = sbase + C::OFF_RAW + slot * C::RAW;
-        const uint32_t rotbase = sbase + C::OFF_ROT + slot * C::ROTB * C::BOX;
-#pragma unroll
-        for (int c = 0; c < C::NB; ++c) {
-          const uint32_t ab = c < rotb ? rotbase + c * C::BOX : rawb + c * C::BOX;
-          const uint32_t qb = sbase + C::OFF_Q + c * C::QSLAB;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(s_tm, smem_desc_sw128(ab + kk * 32, 16, 1024),
-                        smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk, (c | kk) != 0);
-        }
-        mma_commit(&rot_empty[slot]);
-        mma_commit(&s_full[slot]);
-        return true;
-      };
-      auto pv = [&](int i) -> bool {
-        const int slot = i & 1;
-        if (!mbar_wait(&p_full[slot], (i >> 1) & 1, tmo, da.status, abort_flag)) return false;
+        ok = mbar_wait(&p_full[slot], par, tmo, da.status, abort_flag);
+        if (!ok) break;
         tc_fence_after();
         const uint32_t rawb = sbase + C::OFF_RAW + slot * C::RAW;
         const uint32_t pb = sbase + C::OFF_P + slot * C::PSLAB;
@@ -471,19 +536,72 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ss(tmem + C::TM_O + mc * C::NPV,
                         smem_desc_sw128(rawb + 2 * mc * C::BOX + kk * 2048, C::BOX, 1024),
-                        smem_desc_sw128(pb + kk * 32, 16, 1024), idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                        smem_desc_sw128(pb + kk * 32, 16, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&raw_empty[slot]);
-        mma_commit(o_done);
-        return true;
-      };
-      // issue order Q K^T(j), P V(j-1): the S slot of tile j is rewritten by
-      // Q K^T(j+2) only after P V(j), which waited for the softmax of tile j
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = qk(j);
-        if (ok && j >= 1) ok = pv(j - 1);
+        if (j < 24) mark(128 + j);
+        if (j + 2 < ntiles) {
+          ok = mbar_wait(&raw_empty[slot], par, tmo, da.status, abort_flag);
+          if (!ok) break;
+          load(j + 2);
+          issued = j + 3;
+        }
       }
-      if (ok) pv(ntiles - 1);
+      // o_final completes once every P V above has; the TMEM they write
+      // stays allocated until then
       mma_commit(o_final);
+      mbar_wait(o_final, 0, tmo, da.status, nullptr);
+      // let every issued copy land before the CTA can exit
+      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+        mbar_wait(&full[j & 1], (j >> 1) & 1, tmo, da.status, nullptr);
+    }
+  }
+  else {
+    // ------------------------------------------------------------ MMA issuer
+    // S^T = K~ Q~^T: A = key box (K-major, M=64; the side tile's boxes on the
+    // rotated dims), B = Q^T slab (K-major, N=G).  Q K^T(j) waits for its
+    // tile, its side tile, and for the softmax to be done with S(j-2), whose
+    // TMEM slot it rewrites.
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(64, G, false, false);
+      const int rotb = (la.rot + 63) >> 6;
+      bool ok = mbar_wait(q_ready, 0, tmo, da.status, abort_flag);
+      mark(3);
+      // The unrotated dims go first, as soon as the tile has landed; the
+      // rotated ones (from the side tile) once the key prologue is done.
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int slot = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        ok = mbar_wait(&full[slot], par, tmo, da.status, abort_flag) &&
+             (j < 2 || mbar_wait(&p_full[slot], par ^ 1, tmo, da.status, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t s_tm = tmem + (slot ? C::TM_S1 : C::TM_S0);
+        const uint32_t rawb = sbase + C::OFF_RAW + slot * C::RAW;
+        const uint32_t rotbase = sbase + C::OFF_ROT + slot * C::ROTB * C::BOX;
+        for (int c = rotb; c < C::NB; ++c) {
+          const uint32_t ab = rawb + c * C::BOX;
+          const uint32_t qb = sbase + C::OFF_Q + c * C::QSLAB;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(s_tm, smem_desc_sw128(ab + kk * 32, 16, 1024),
+                        smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk, (c > rotb || kk > 0) ? 1u : 0u);
+        }
+        if (j < 24) mark(56 + j);
+        ok = mbar_wait(&rot_full[slot], par, tmo, da.status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        for (int c = 0; c < rotb; ++c) {
+          const uint32_t ab = rotbase + c * C::BOX;
+          const uint32_t qb = sbase + C::OFF_Q + c * C::QSLAB;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(s_tm, smem_desc_sw128(ab + kk * 32, 16, 1024),
+                        smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk,
+                        (rotb < C::NB || c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&rot_empty[slot]);
+        mma_commit(&s_full[slot]);
+      }
       // every MMA issued above has completed before TMEM is released
       mma_commit(drain);
       mbar_wait(drain, 0, tmo, da.status, nullptr);
@@ -496,6 +614,7 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  if (threadIdx.x == 0) mark(5);
 }
 
 template <int D, int G>

@@ -351,6 +351,8 @@ int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf1
   da.B = batch;
   da.max_len = max_len;
   da.status = static_cast<uint32_t*>(workspace);
+  da.trace = static_cast<unsigned long long*>(g_trace_buf);
+  da.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
   cudaError_t e = gattn::launch_decode_split(da, la, s);

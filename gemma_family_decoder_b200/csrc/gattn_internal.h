@@ -49,6 +49,8 @@ struct DecodeArgs {
   float* part_o;   // [B][H][nsplit][D]
   float* part_ml;  // [B][H][nsplit][2]
   uint32_t* status;
+  unsigned long long* trace = nullptr;  // optional per-CTA timeline (tensor-core kernel)
+  size_t trace_bytes = 0;
 };
 void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk);
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
