@@ -324,50 +324,66 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   } else if (warp == 4) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      int n = 0;
       mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
       for (int sl = 0; sl < D / 64; ++sl)
         tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
-      auto load = [&](const CUtensorMap* tm, int d0, int key0) -> bool {
-        const int st = n % C::NSTAGE;
-        const uint32_t par = ((n / C::NSTAGE) & 1) ^ 1;
-        if (!mbar_wait(&empty[st], par, tmo, P.status, abort_flag)) return false;
-        mbar_arrive_expect_tx(&full[st], C::SLAB_KV);
-        tma_load_4d(smem + C::OFF_RING + st * C::SLAB_KV, tm, &full[st], d0, kvh, key0, b);
-        ++n;
+      // Each key tile (KCH boxes, slots [0, KCH)) and each value tile (VCH
+      // boxes, slots [KCH, NSTAGE)) lands under one barrier phase: a phase
+      // per box would cap this thread's copy stream far below the L2 rate.
+      uint64_t* kf = &full[0];
+      uint64_t* ke = &empty[0];
+      uint64_t* vf = &full[C::KCH];
+      uint64_t* ve = &empty[C::KCH];
+      auto load_k = [&](int j) -> bool {
+        if (!mbar_wait(ke, (j & 1) ^ 1, tmo, P.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(kf, C::KCH * C::SLAB_KV);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(smem + C::OFF_RING + c * C::SLAB_KV, &P.tm_k, kf, c * 64, kvh, tile_key(j), b);
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        if (!mbar_wait(ve, (j & 1) ^ 1, tmo, P.status, abort_flag)) return false;
+        mbar_arrive_expect_tx(vf, C::VCH * C::SLAB_KV);
+        for (int c = 0; c < C::VCH; ++c)
+          tma_load_4d(smem + C::OFF_RING + (C::KCH + c) * C::SLAB_KV, &P.tm_v, vf, dv_lo + c * 64, kvh,
+                      tile_key(j), b);
         return true;
       };
       // same order as the MMA issuer consumes them: K(j) then V(j-1)
       bool ok = true;
+      int lk = -1, lv = -1;  // last key / value tile issued
       for (int j = 0; j < ntiles && ok; ++j) {
-        const int key0 = tile_key(j);
-        for (int c = 0; c < C::KCH && ok; ++c) ok = load(&P.tm_k, c * 64, key0);
-        for (int c = 0; c < C::VCH && ok && j >= 1; ++c) ok = load(&P.tm_v, dv_lo + c * 64, tile_key(j - 1));
+        ok = load_k(j);
+        if (ok) lk = j;
+        if (ok && j >= 1) ok = load_v(j - 1);
+        if (ok && j >= 1) lv = j - 1;
       }
-      for (int c = 0; c < C::VCH && ok; ++c) ok = load(&P.tm_v, dv_lo + c * 64, tile_key(ntiles - 1));
+      if (ok && load_v(ntiles - 1)) lv = ntiles - 1;
       // let every issued copy land before the CTA can exit
       mbar_wait(q_full, 0, tmo, P.status, nullptr);
-      for (int i = n - C::NSTAGE < 0 ? 0 : n - C::NSTAGE; i < n; ++i)
-        mbar_wait(&full[i % C::NSTAGE], (i / C::NSTAGE) & 1, tmo, P.status, nullptr);
+      if (lk >= 0) mbar_wait(kf, lk & 1, tmo, P.status, nullptr);
+      if (lv >= 0) mbar_wait(vf, lv & 1, tmo, P.status, nullptr);
     }
   } else {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
-      int n = 0;
       bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
       mark(3);
       tc_fence_after();
+      uint64_t* kf = &full[0];
+      uint64_t* ke = &empty[0];
+      uint64_t* vf = &full[C::KCH];
+      uint64_t* ve = &empty[C::KCH];
       auto qk = [&](int j) -> bool {
         const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
+        if (!mbar_wait(kf, j & 1, tmo, P.status, abort_flag)) return false;
+        if (j == 0) mark(6);
+        tc_fence_after();
         for (int c = 0; c < C::KCH; ++c) {
-          const int st = n % C::NSTAGE;
-          if (!mbar_wait(&full[st], (n / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
-          if (n == 0) mark(6);
-          tc_fence_after();
-          const uint32_t kb = sbase + C::OFF_RING + st * C::SLAB_KV;
+          const uint32_t kb = sbase + C::OFF_RING + c * C::SLAB_KV;
           const uint32_t qb = sbase + C::OFF_Q + c * C::SLAB128;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
@@ -375,9 +391,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
             const uint64_t a = smem_desc_sw128(qb + kk * 32, 16, 1024);
             mma_bf16_ss(s_tm, a, bd, idesc_qk, (c | kk) != 0);
           }
-          mma_commit(&empty[st]);
-          ++n;
         }
+        mma_commit(ke);
         mma_commit(&s_full[j & 1]);
         if (j < 120) mark(248 + j);
         return true;
@@ -385,14 +400,9 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, tmo, P.status, abort_flag)) return false;
         const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
-        // the VCH value boxes sit in VCH consecutive slots (tiles are 4-slot aligned)
-        const int st0 = n % C::NSTAGE;
-        for (int c = 0; c < C::VCH; ++c) {
-          const int st = st0 + c;
-          if (!mbar_wait(&full[st], ((n + c) / C::NSTAGE) & 1, tmo, P.status, abort_flag)) return false;
-        }
+        if (!mbar_wait(vf, i & 1, tmo, P.status, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vb = sbase + C::OFF_RING + st0 * C::SLAB_KV;
+        const uint32_t vb = sbase + C::OFF_RING + C::KCH * C::SLAB_KV;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // 16 keys x 256 value dims, MN-major: key rows 128 B apart, 8-row groups
@@ -400,8 +410,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
           mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        for (int c = 0; c < C::VCH; ++c) mma_commit(&empty[st0 + c]);
-        n += C::VCH;
+        mma_commit(ve);
         mma_commit(o_done);
         if (i < 120) mark(368 + i);
         return true;
