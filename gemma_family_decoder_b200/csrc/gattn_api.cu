@@ -227,9 +227,10 @@ size_t gattn_prefill_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t
   gattn::LayerArgs la;
   if (resolve(cfg, &la, false) != GATTN_OK || batch < 0 || seq_len < 0) return 0;
   size_t bytes = kStatusBytes;
-  if (prefill_needs_kprep(la))
+  if (prefill_needs_kprep(la))  // transformed keys, then transformed queries
     bytes = round_up(bytes, 1024) +
-            static_cast<size_t>(batch) * seq_len * la.Hkv * la.D * sizeof(uint16_t);
+            round_up(static_cast<size_t>(batch) * seq_len * la.Hkv * la.D * sizeof(uint16_t), 1024) +
+            static_cast<size_t>(batch) * seq_len * la.H * la.D * sizeof(uint16_t);
   return bytes;
 }
 
@@ -264,15 +265,22 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   uint32_t* status = static_cast<uint32_t*>(workspace);
   const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(k);
   const __nv_bfloat16* kt = kb;
-  if (prefill_needs_kprep(la)) {
-    __nv_bfloat16* ktw = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) +
-                                                          round_up(kStatusBytes, 1024));
-    cudaError_t e = gattn::launch_kprep(kb, positions, ktw, batch, seq_len, la, status, s);
-    if (e != cudaSuccess) return fail_cuda(e, "key prologue launch");
+  const __nv_bfloat16* qt = reinterpret_cast<const __nv_bfloat16*>(q);
+  const bool prep = prefill_needs_kprep(la);
+  if (prep) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    __nv_bfloat16* ktw = reinterpret_cast<__nv_bfloat16*>(ws + round_up(kStatusBytes, 1024));
+    __nv_bfloat16* qtw = reinterpret_cast<__nv_bfloat16*>(
+        ws + round_up(kStatusBytes, 1024) +
+        round_up(static_cast<size_t>(batch) * seq_len * la.Hkv * la.D * sizeof(uint16_t), 1024));
+    cudaError_t e = gattn::launch_qkprep(qt, kb, positions, qtw, ktw, batch, seq_len, la, status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "query/key prologue launch");
     kt = ktw;
+    qt = qtw;
   }
   gattn::PrefillArgs pa;
-  pa.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  pa.q = qt;
+  pa.q_prepared = prep ? 1 : 0;
   pa.kt = kt;
   pa.v = la.k_eq_v ? kb : reinterpret_cast<const __nv_bfloat16*>(v_or_null);
   pa.positions = positions;

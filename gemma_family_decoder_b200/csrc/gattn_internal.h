@@ -33,9 +33,11 @@ struct LayerArgs {
 cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim, int max_pos,
                               cudaStream_t s);
 
-// k~ = RoPE(RMSNorm(k)) for every (b, s, kv head) row, bf16 out, same layout.
-cudaError_t launch_kprep(const __nv_bfloat16* k, const int* positions, __nv_bfloat16* kt,
-                         int B, int S, const LayerArgs& la, uint32_t* status, cudaStream_t s);
+// q~ = RoPE(RMSNorm(q)) for every (b, s, head) row and k~ = RoPE(RMSNorm(k))
+// for every (b, s, kv head) row, bf16 out, same layouts, in one launch.
+cudaError_t launch_qkprep(const __nv_bfloat16* q, const __nv_bfloat16* k, const int* positions,
+                          __nv_bfloat16* qt, __nv_bfloat16* kt, int B, int S, const LayerArgs& la,
+                          uint32_t* status, cudaStream_t s);
 
 // Split-KV decode: partials (m, l, O) per (b, h, split) then the merge.
 struct DecodeArgs {
@@ -62,7 +64,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStre
 
 // Prefill on tcgen05 tensor cores.
 struct PrefillArgs {
-  const __nv_bfloat16* q;
+  const __nv_bfloat16* q;   // queries; already normed and rotated when q_prepared
+  int q_prepared;
   const __nv_bfloat16* kt;  // transformed keys (or raw k when no transform applies)
   const __nv_bfloat16* v;   // values (raw k when k_eq_v)
   const int* positions;

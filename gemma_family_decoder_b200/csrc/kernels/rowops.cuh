@@ -98,6 +98,62 @@ __device__ __forceinline__ void transform_row(float (&x)[NCH][8], int lane, int 
   }
 }
 
+// The same RMSNorm + RoPE with the (cos, sin) of each of the lane's elements
+// given (cs[i][e] for dim 8 (lane + 32 i) + e, read only on rotated dims):
+// rows that share a position share the angles.
+template <int NCH>
+__device__ __forceinline__ void transform_row_cs(float (&x)[NCH][8], int lane, const LayerArgs& la,
+                                                 const float* w, const float2 (&cs)[NCH][8]) {
+  constexpr int D = NCH * 256;
+  if (la.qk_norm) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += x[i][e] * x[i][e];
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / static_cast<float>(D) + la.eps);
+    const float off = la.qk_norm == 1 ? 1.f : 0.f;
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = lane + 32 * i;
+      const float4 g0 = __ldg(w4 + 2 * c), g1 = __ldg(w4 + 2 * c + 1);
+      x[i][0] *= r * (g0.x + off); x[i][1] *= r * (g0.y + off);
+      x[i][2] *= r * (g0.z + off); x[i][3] *= r * (g0.w + off);
+      x[i][4] *= r * (g1.x + off); x[i][5] *= r * (g1.y + off);
+      x[i][6] *= r * (g1.z + off); x[i][7] *= r * (g1.w + off);
+    }
+  }
+  if (la.rot > 0) {
+    const int half = la.rot >> 1;
+    const int h16 = la.rot >> 4;
+    float pr[NCH][8];
+    if (h16 < 32) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = __shfl_xor_sync(0xffffffffu, x[i][e], h16);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[i][e] = x[NCH - 1 - i][e];
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = lane + 32 * i;
+      if (8 * c < la.rot) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bool first = 8 * c + e < half;
+          x[i][e] = first ? x[i][e] * cs[i][e].x - pr[i][e] * cs[i][e].y
+                          : x[i][e] * cs[i][e].x + pr[i][e] * cs[i][e].y;
+        }
+      }
+    }
+  }
+}
 
 // 8 floats <-> 8 packed bf16 (16 bytes)
 __device__ __forceinline__ void unpack8(const uint4 u, float (&x)[8]) {

@@ -70,6 +70,7 @@ struct PrefillKParams {
   uint32_t* status;
   uint64_t timeout_ns;
   int B, S, nqt, dv_splits;
+  int q_prepared;
   LayerArgs la;
   unsigned long long* trace;  // optional per-CTA event times (kTraceSlots each), or null
   int trace_ctas;
@@ -182,8 +183,9 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
 
-    // query prologue in place, thread t on row t; RoPE angles computed, not read
-    if (ok && valid && (la.rot > 0 || la.qk_norm)) {
+    // query prologue in place, thread t on row t; RoPE angles computed, not
+    // read (only when the queries were not transformed by the prologue kernel)
+    if (ok && valid && !P.q_prepared && (la.rot > 0 || la.qk_norm)) {
       int pos = la.rot > 0 ? __ldg(P.positions + static_cast<size_t>(b) * S + qi) : 0;
       if (la.rot > 0 && (pos < 0 || pos >= la.rope_max_pos)) {
         flag_status(P.status, kStatusBounds);
@@ -448,6 +450,7 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
       !encode_tmap_bshd(&P.tm_o, pa.out, pa.B, pa.S, la.H, D, C::BM))
     return cudaErrorInvalidValue;
   P.positions = pa.positions;
+  P.q_prepared = pa.q_prepared;
   P.status = pa.status;
   P.timeout_ns = pa.timeout_ns;
   P.B = pa.B;

@@ -45,42 +45,100 @@ cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim,
 }
 
 // ---------------------------------------------------------------------------
-// Key prologue for prefill: one warp per (b, s, kv head) row.
+// Query and key prologue for prefill, elementwise.  TPR = D/16 threads (a 16-
+// or 32-lane group) serve one token (b, s); thread i owns two 8-dim chunks of
+// every row of the token: a RoPE pair (chunk i and chunk i + R/16) when
+// i < R/16, else two unrotated chunks.  It reads the token's position and
+// its (cos, sin) from the RoPE table once, then walks the token's H query
+// rows (query gain) and Hkv key rows (key gain), RB rows at a time with
+// their loads issued together; outputs keep the input layouts.
 // ---------------------------------------------------------------------------
-template <int NCH>
-__global__ void __launch_bounds__(256) kprep_kernel(const bf16* __restrict__ k,
-                                                    const int* __restrict__ positions,
-                                                    bf16* __restrict__ kt, long long rows,
-                                                    LayerArgs la, uint32_t* status) {
-  constexpr int D = NCH * 256;
-  const int lane = threadIdx.x & 31;
-  const long long row = blockIdx.x * 8LL + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const long long bs = row / la.Hkv;
-  const int pos = positions ? __ldg(positions + bs) : 0;
-  float x[NCH][8];
-  load_row<NCH>(k + row * D, lane, x);
-  transform_row<NCH>(x, lane, pos, la, la.k_norm_w, status);
-  uint4* dst = reinterpret_cast<uint4*>(kt + row * D);
+template <int TPR, int RB>
+__global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
+                                                     const int* __restrict__ positions,
+                                                     bf16* __restrict__ qt, bf16* __restrict__ kt,
+                                                     long long tokens, LayerArgs la, uint32_t* status) {
+  constexpr int D = TPR * 16;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long bs = gid / TPR;
+  const int i = static_cast<int>(gid % TPR);
+  if (bs >= tokens) return;  // whole groups leave together (TPR divides 32)
+  const unsigned gmask = TPR == 32 ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
+  const int h8 = la.rot >> 4;  // chunks in half the rotated slice
+  const bool rotated = i < h8;
+  const int c0 = rotated ? i : 2 * h8 + 2 * (i - h8);
+  const int c1 = rotated ? i + h8 : c0 + 1;
+  float4 cs[4];  // (cos, sin) of pairs 8i .. 8i+7, two pairs per float4
+  if (rotated) {
+    const int pos = checked_pos(positions ? __ldg(positions + bs) : 0, la, status);
+    const float4* trow = reinterpret_cast<const float4*>(la.rope_tab + static_cast<size_t>(pos) * (la.rot >> 1)) + 4 * i;
 #pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    uint4 u;
-    u.x = pack_bf16x2(x[i][0], x[i][1]);
-    u.y = pack_bf16x2(x[i][2], x[i][3]);
-    u.z = pack_bf16x2(x[i][4], x[i][5]);
-    u.w = pack_bf16x2(x[i][6], x[i][7]);
-    dst[lane + 32 * i] = u;
+    for (int e = 0; e < 4; ++e) cs[e] = __ldg(trow + e);
+  }
+  const float off = la.qk_norm == 1 ? 1.f : 0.f;
+  const int nrows = la.H + la.Hkv;
+  for (int r0 = 0; r0 < nrows; r0 += RB) {
+    uint4 u0[RB], u1[RB];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int r = r0 + u;
+      if (r < nrows) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            r < la.H ? q + (bs * la.H + r) * D : k + (bs * la.Hkv + (r - la.H)) * D);
+        u0[u] = __ldg(src + c0);
+        u1[u] = __ldg(src + c1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int r = r0 + u;
+      if (r >= nrows) break;  // uniform over the group
+      const bool is_q = r < la.H;
+      float x0[8], x1[8];
+      unpack8(u0[u], x0);
+      unpack8(u1[u], x1);
+      if (la.qk_norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x0[e], x0[e], fmaf(x1[e], x1[e], ss));
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gmask, ss, o);
+        const float rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
+        const float4* w4 = reinterpret_cast<const float4*>(is_q ? la.q_norm_w : la.k_norm_w);
+        const float4 a0 = __ldg(w4 + 2 * c0), a1 = __ldg(w4 + 2 * c0 + 1);
+        const float4 b0 = __ldg(w4 + 2 * c1), b1 = __ldg(w4 + 2 * c1 + 1);
+        x0[0] *= rn * (a0.x + off); x0[1] *= rn * (a0.y + off); x0[2] *= rn * (a0.z + off); x0[3] *= rn * (a0.w + off);
+        x0[4] *= rn * (a1.x + off); x0[5] *= rn * (a1.y + off); x0[6] *= rn * (a1.z + off); x0[7] *= rn * (a1.w + off);
+        x1[0] *= rn * (b0.x + off); x1[1] *= rn * (b0.y + off); x1[2] *= rn * (b0.z + off); x1[3] *= rn * (b0.w + off);
+        x1[4] *= rn * (b1.x + off); x1[5] *= rn * (b1.y + off); x1[6] *= rn * (b1.z + off); x1[7] *= rn * (b1.w + off);
+      }
+      if (rotated) {
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const float4 c = cs[e / 2];
+          const float a = x0[e], bb = x1[e], a2 = x0[e + 1], b2 = x1[e + 1];
+          x0[e] = a * c.x - bb * c.y;
+          x1[e] = bb * c.x + a * c.y;
+          x0[e + 1] = a2 * c.z - b2 * c.w;
+          x1[e + 1] = b2 * c.z + a2 * c.w;
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(is_q ? qt + (bs * la.H + r) * D : kt + (bs * la.Hkv + (r - la.H)) * D);
+      dst[c0] = pack8(x0);
+      dst[c1] = pack8(x1);
+    }
   }
 }
 
-cudaError_t launch_kprep(const bf16* k, const int* positions, bf16* kt, int B, int S,
-                         const LayerArgs& la, uint32_t* status, cudaStream_t s) {
-  const long long rows = static_cast<long long>(B) * S * la.Hkv;
-  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+cudaError_t launch_qkprep(const bf16* q, const bf16* k, const int* positions, bf16* qt, bf16* kt,
+                          int B, int S, const LayerArgs& la, uint32_t* status, cudaStream_t s) {
+  const long long tokens = static_cast<long long>(B) * S;
+  const long long threads = tokens * (la.D / 16);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
   if (la.D == 256)
-    kprep_kernel<1><<<blocks, 256, 0, s>>>(k, positions, kt, rows, la, status);
+    qkprep_kernel<16, 3><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status);
   else
-    kprep_kernel<2><<<blocks, 256, 0, s>>>(k, positions, kt, rows, la, status);
+    qkprep_kernel<32, 3><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status);
   return cudaGetLastError();
 }
 
