@@ -280,10 +280,8 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   }
   gattn::PrefillArgs pa;
   pa.q = qt;
-  pa.q_prepared = prep ? 1 : 0;
   pa.kt = kt;
   pa.v = la.k_eq_v ? kb : reinterpret_cast<const __nv_bfloat16*>(v_or_null);
-  pa.positions = positions;
   pa.out = reinterpret_cast<__nv_bfloat16*>(out);
   pa.B = batch;
   pa.S = seq_len;

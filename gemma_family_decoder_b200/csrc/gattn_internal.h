@@ -64,11 +64,9 @@ cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStre
 
 // Prefill on tcgen05 tensor cores.
 struct PrefillArgs {
-  const __nv_bfloat16* q;   // queries; already normed and rotated when q_prepared
-  int q_prepared;
+  const __nv_bfloat16* q;   // transformed queries (or raw q when no transform applies)
   const __nv_bfloat16* kt;  // transformed keys (or raw k when no transform applies)
   const __nv_bfloat16* v;   // values (raw k when k_eq_v)
-  const int* positions;
   __nv_bfloat16* out;
   int B, S;
   uint32_t* status;

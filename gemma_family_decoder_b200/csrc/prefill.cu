@@ -1,23 +1,25 @@
 // Prefill self-attention on the sm_100a tensor cores (tcgen05 + TMA + TMEM).
 //
-// One CTA computes a 128-query tile of one head (and, for head_dim 512, one
-// 256-wide half of the value dims).  Warp roles:
-//   warps 0-3  query prologue: the raw Q tile arrives by TMA and each thread
-//              applies QK-norm + RoPE to its own row in shared memory; then per
-//              KV tile: S from TMEM -> scale (and softcap) -> causal/window mask
-//              on boundary tiles only -> online softmax with lazy rescale ->
-//              P (bf16) written back into the same TMEM columns; finally
-//              O / l -> bf16 -> shared memory -> TMA store.
-//   warp 4     TMA producer: the Q tile, then transformed-key tiles and value
-//              tiles, one 64-dim box at a time, into a ring of box-sized slots
-//              (about one key tile plus one value tile of look-ahead).
+// A persistent kernel: one CTA per SM takes work items in turn, an item being
+// a 128-query tile of one head (and, for head_dim 512, one 256-wide half of
+// the value dims), heaviest items first.  The queries arrive already normed
+// and rotated (the prologue kernel).  Warp roles:
+//   warps 0-3  per KV tile: S from TMEM -> scale (and softcap) -> causal/window
+//              mask on boundary tiles only -> online softmax with lazy rescale
+//              -> P (bf16) written back into the same TMEM columns; at the
+//              end of an item, O / l -> bf16 straight to global memory.
+//   warp 4     TMA producer: per item the first key tile, the Q tile (once the
+//              previous item's last Q K^T is done with the buffer), then key
+//              and value tiles, each under one barrier phase, into a ring of
+//              one key tile and one value tile.
 //   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM slot, then
 //              O += P V with P read from that slot, into the TMEM accumulator.
 // Because P lives in the S slot, the softmax of tile j+1 never waits for the
 // P V product of tile j (it waits only in the rare case that O must be
 // rescaled), and the tensor core runs Q K^T of tile j+1 while the softmax of
-// tile j is still being computed.
-// KV tiles entirely outside the causal window are never visited.
+// tile j is still being computed.  Barrier phases count tiles and items over
+// the whole run of a CTA, so the next item's loads start while the current
+// one finishes.  KV tiles entirely outside the causal window are never visited.
 //
 // Layer definition: KerasFormers "Gemma 4" (What changed: plain-weight RMSNorm,
 // partial rotation, K=V global layers), KerasFormers "Gemma 3" (What changed:
@@ -45,7 +47,7 @@ struct PrefillShape {
   // ring slots: a multiple of 4 so that every 4-slot value tile is contiguous
   static constexpr int NSTAGE = ((227 * 1024 - Q_BYTES - 2048) / SLAB_KV) / 4 * 4;
   static constexpr int OFF_RING = Q_BYTES;
-  static constexpr int OFF_Q = 0;  // Q tile (and later the O tile)
+  static constexpr int OFF_Q = 0;
   static constexpr int OFF_BAR = OFF_RING + NSTAGE * SLAB_KV;
   static constexpr int NBAR = 2 * NSTAGE + 10;
   static_assert(NSTAGE >= KCH + VCH, "ring must hold a key tile and a value tile");
@@ -58,29 +60,28 @@ struct PrefillShape {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(TM_S1 + BN <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(Q_BYTES >= BM * DV * 2, "the output tile reuses the Q tile's shared memory");
+  static_assert(NSTAGE == KCH + VCH, "the ring is one key tile and one value tile");
 };
 
 struct PrefillKParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_o;
-  const int* positions;
+  __nv_bfloat16* out;
   uint32_t* status;
   uint64_t timeout_ns;
   int B, S, nqt, dv_splits;
-  int q_prepared;
   LayerArgs la;
   unsigned long long* trace;  // optional per-CTA event times (kTraceSlots each), or null
   int trace_ctas;
 };
 
-// Optional timeline of one CTA (debug aid, off unless a trace buffer is set):
-// [0] start time (ns), [1] SM id, [2] KV tiles, [3] Q ready at the MMA warp,
-// [4] epilogue start, [5] end, [6] first key box landed, then per KV tile j
-// (j < 120): [8+j] S(j) seen by the softmax, [128+j] P(j) written,
-// [248+j] Q K^T(j) issued, [368+j] P V(j) issued; times relative to [0].
+// Optional timeline of one CTA's first item (debug aid, off unless a trace
+// buffer is set): [0] start time (ns), [1] SM id, [2] KV tiles, [3] Q landed
+// at the MMA warp, [4] epilogue start, [5] end of the CTA, [6] first key tile
+// landed, [7] items of the CTA, then per KV tile j (j < 120): [8+j] S(j) seen
+// by the softmax, [128+j] P(j) written, [248+j] Q K^T(j) issued, [368+j]
+// P V(j) issued; times relative to [0].
 constexpr int kTraceSlots = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -92,57 +93,73 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + C::NSTAGE;
-  uint64_t* s_full = bars + 2 * C::NSTAGE;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* q_ready = o_done + 1;
-  uint64_t* drain = q_ready + 1;
-  uint64_t* q_full = drain + 1;
-  uint64_t* o_final = q_full + 1;
+  uint64_t* kf = bars;          // key tile landed (one phase per KV tile)
+  uint64_t* ke = bars + 1;      // Q K^T done with the key tile
+  uint64_t* vf = bars + 2;      // value tile landed
+  uint64_t* ve = bars + 3;      // P V done with the value tile
+  uint64_t* s_full = bars + 4;  // [2] S ready in its TMEM slot
+  uint64_t* p_full = bars + 6;  // [2] P written over it (128 arrivals)
+  uint64_t* o_done = bars + 8;  // one phase per P V
+  uint64_t* q_full = bars + 9;  // Q tile landed (one phase per item)
+  uint64_t* q_empty = bars + 10;  // the item's last Q K^T is done with the Q tile
+  uint64_t* o_final = bars + 11;  // the item's last P V is done
+  uint64_t* o_empty = bars + 12;  // the softmax has read the item's O (128 arrivals)
+  uint64_t* drain = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const LayerArgs& la = P.la;
   const int H = la.H, S = P.S;
-  // work item: heaviest query tiles first
-  int idx = blockIdx.x;
-  const int per_qt = P.B * H * P.dv_splits;
-  const int qt = P.nqt - 1 - idx / per_qt;
-  idx %= per_qt;
-  const int dvs = idx % P.dv_splits;
-  idx /= P.dv_splits;
-  const int h = idx % H;
-  const int b = idx / H;
-  const int kvh = h / la.G;
-  const int q0 = qt * C::BM;
-  const int dv_lo = dvs * C::DV;
-  const int kv_hi = min(S, q0 + C::BM);
-  const int kv_lo = la.window > 0 ? max(0, q0 - la.window + 1) : 0;
-  const int k_first = (kv_lo / BN) * BN;
-  const int ntiles = (kv_hi - k_first + BN - 1) / BN;
-  // KV tiles are visited starting at a tile that differs between the CTAs
-  // working on one sequence at once, so they do not all read the same L2 lines
-  // together (the online softmax is independent of the visiting order)
-  const int rot = ntiles > 1 ? (h * 7 + dvs * 3 + b * 5 + qt) % ntiles : 0;
-  auto tile_key = [&](int j) { return k_first + ((j + rot) % ntiles) * BN; };
+  const int nitems = P.nqt * P.B * H * P.dv_splits;
+  // work item `it`, heaviest query tiles first
+  struct Item {
+    int qt, dvs, h, b, kvh, q0, dv_lo, k_first, ntiles, rot;
+  };
+  auto item_of = [&](int it) {
+    Item w;
+    const int per_qt = P.B * H * P.dv_splits;
+    w.qt = P.nqt - 1 - it / per_qt;
+    int idx = it % per_qt;
+    w.dvs = idx % P.dv_splits;
+    idx /= P.dv_splits;
+    w.h = idx % H;
+    w.b = idx / H;
+    w.kvh = w.h / la.G;
+    w.q0 = w.qt * C::BM;
+    w.dv_lo = w.dvs * C::DV;
+    const int kv_hi = min(S, w.q0 + C::BM);
+    const int kv_lo = la.window > 0 ? max(0, w.q0 - la.window + 1) : 0;
+    w.k_first = (kv_lo / BN) * BN;
+    w.ntiles = (kv_hi - w.k_first + BN - 1) / BN;
+    // KV tiles are visited starting at a tile that differs between the items
+    // working on one sequence at once, so they do not all read the same L2
+    // lines together (the online softmax is independent of the visiting order)
+    w.rot = w.ntiles > 1 ? (w.h * 7 + w.dvs * 3 + w.b * 5 + w.qt) % w.ntiles : 0;
+    return w;
+  };
+  auto tile_key = [&](const Item& w, int j) { return w.k_first + ((j + w.rot) % w.ntiles) * BN; };
+  // This CTA's items: round r gives it item r*G + c, or r*G + G-1-c on odd
+  // rounds, so that the heaviest-first items spread evenly over the CTAs.
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int nrounds = (nitems + G - 1) / G;
+  auto item_at = [&](int r) { return r * G + ((r & 1) ? G - 1 - cta : cta); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NSTAGE; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
     }
+    mbar_init(kf, 1);
+    mbar_init(ke, 1);
+    mbar_init(vf, 1);
+    mbar_init(ve, 1);
     mbar_init(o_done, 1);
-    mbar_init(q_ready, 128);
-    mbar_init(drain, 1);
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     mbar_init(o_final, 1);
+    mbar_init(o_empty, 128);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -150,7 +167,6 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     tma_prefetch_desc(&P.tm_q);
     tma_prefetch_desc(&P.tm_k);
     tma_prefetch_desc(&P.tm_v);
-    tma_prefetch_desc(&P.tm_o);
   }
   if (warp == 5) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -172,217 +188,214 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
     trace[0] = t_start;
     trace[1] = smid;
-    trace[2] = ntiles;
+    int n = 0;
+    for (int r = 0; r < nrounds; ++r) n += item_at(r) < nitems;
+    trace[2] = item_of(item_at(0)).ntiles;
+    trace[7] = n;
   }
 
   if (warp < 4) {
     // ------------------------------------------------------------------ softmax
     const int t = threadIdx.x;
-    const int qi = q0 + t;
-    const bool valid = qi < S;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, tmo, P.status, abort_flag));
-
-    // query prologue in place, thread t on row t; RoPE angles computed, not
-    // read (only when the queries were not transformed by the prologue kernel)
-    if (ok && valid && !P.q_prepared && (la.rot > 0 || la.qk_norm)) {
-      int pos = la.rot > 0 ? __ldg(P.positions + static_cast<size_t>(b) * S + qi) : 0;
-      if (la.rot > 0 && (pos < 0 || pos >= la.rope_max_pos)) {
-        flag_status(P.status, kStatusBounds);
-        pos = pos < 0 ? 0 : la.rope_max_pos - 1;
-      }
-      const float rn = la.qk_norm ? rsqrtf(tile_row_sumsq(smem + C::OFF_Q, C::SLAB128, t, 0, D / 8) /
-                                               static_cast<float>(D) + la.eps)
-                                  : 1.f;
-      tile_row_prologue(smem + C::OFF_Q, C::SLAB128, t, pos, la, rn, 0, la.rot >> 4, la.rot >> 3, D / 8);
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(q_ready);
-
-    // main loop over KV tiles
     const float sl2 = la.scale_log2;
     const float kcap = CAP ? la.scale / la.softcap : 0.f;
     const float cap_l2 = CAP ? la.softcap * kLog2e : 0.f;
     const int W = la.window;
-    float m = -INFINITY, l = 0.f;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, tmo, P.status, abort_flag));
-      if (!ok) break;
-      if (t == 0 && j < 120) mark(8 + j);
-      tc_fence_after();
-      const uint32_t scol = tmem + lane_off + ((j & 1) ? C::TM_S1 : C::TM_S0);
-      uint32_t rr[BN / 32][32];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
-      tmem_wait_ld();
-
-      const int key0 = tile_key(j);
-      const bool full_tile = (key0 + BN - 1 <= q0) && (q0 + C::BM <= S) &&
-                             (W <= 0 || (q0 + C::BM - 1) - key0 < W);
-      float x[BN];
-#pragma unroll
-      for (int i = 0; i < BN; ++i) {
-        const float s = __uint_as_float(rr[i >> 5][i & 31]);
-        x[i] = CAP ? cap_l2 * tanh_fast(s * kcap) : s;
-      }
-      if (!full_tile) {
-        const int hi = valid ? qi - key0 : -1;            // visible iff i <= hi
-        const int lo = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
-#pragma unroll
-        for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
-      }
-      float mxa[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) mxa[a] = x[a];
-#pragma unroll
-      for (int i = 8; i < BN; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], x[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                             fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
-      const float m_tile = CAP ? mx : mx * sl2;   // running max in log2 units
-      const float m_new = fmaxf(m, m_tile);
-      float alpha = 1.f;
-      bool rescale = false;
-      float m_use = m;
-      if (m_new > m + 8.f) {
-        m_use = m_new;
-        rescale = (m != -INFINITY);
-        alpha = rescale ? ex2(m - m_new) : 0.f;
-      }
-      const float mu = (m_use == -INFINITY) ? 0.f : m_use;
-      float rsa[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) rsa[a] = 0.f;
-      uint32_t pk[BN / 64][32];
-#pragma unroll
-      for (int i = 0; i < BN; i += 2) {
-        const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
-        const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
-        rsa[(i >> 1) & 7] += p0 + p1;
-        pk[i >> 6][(i >> 1) & 31] = pack_bf16x2(p0, p1);
-      }
-      const float rs = ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
-      // P (bf16 pairs) over the first BN/2 columns of this S slot
-#pragma unroll
-      for (int c = 0; c < BN / 64; ++c) tmem_st32(scol + c * 32, pk[c]);
-      // O must hold P V of every earlier tile before it is rescaled; that is
-      // the only case in which the softmax waits for the tensor core.  Seeing
-      // S(j) implies P V(j-2) is complete (it was issued before Q K^T(j)), so
-      // o_done is at most one phase behind and its parity wait is exact.
-      if (__any_sync(0xffffffffu, rescale) && j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, P.status, abort_flag));
+    bool ok = true;
+    int T0 = 0;  // KV tiles of this CTA's earlier items
+    for (int r = 0, I = 0; r < nrounds && ok; ++r) {
+      const int it = item_at(r);
+      if (it >= nitems) continue;
+      const Item w = item_of(it);
+      const int qi = w.q0 + t;
+      const bool valid = qi < S;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < w.ntiles && ok; ++j) {
+        const int T = T0 + j;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[T & 1], (T >> 1) & 1, tmo, P.status, abort_flag));
         if (!ok) break;
+        if (t == 0 && I == 0 && j < 120) mark(8 + j);
         tc_fence_after();
-        const float f = rescale ? alpha : 1.f;
+        const uint32_t scol = tmem + lane_off + ((T & 1) ? C::TM_S1 : C::TM_S0);
+        uint32_t rr[BN / 32][32];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) tmem_ld32(scol + c * 32, rr[c]);
+        tmem_wait_ld();
+
+        const int key0 = tile_key(w, j);
+        const bool full_tile = (key0 + BN - 1 <= w.q0) && (w.q0 + C::BM <= S) &&
+                               (W <= 0 || (w.q0 + C::BM - 1) - key0 < W);
+        float x[BN];
+#pragma unroll
+        for (int i = 0; i < BN; ++i) {
+          const float sv = __uint_as_float(rr[i >> 5][i & 31]);
+          x[i] = CAP ? cap_l2 * tanh_fast(sv * kcap) : sv;
+        }
+        if (!full_tile) {
+          const int hi = valid ? qi - key0 : -1;            // visible iff i <= hi
+          const int lo = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
+#pragma unroll
+          for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
+        }
+        float mxa[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mxa[a] = x[a];
+#pragma unroll
+        for (int i = 8; i < BN; ++i) mxa[i & 7] = fmaxf(mxa[i & 7], x[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                               fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7])));
+        const float m_tile = CAP ? mx : mx * sl2;   // running max in log2 units
+        const float m_new = fmaxf(m, m_tile);
+        float alpha = 1.f;
+        bool rescale = false;
+        float m_use = m;
+        if (m_new > m + 8.f) {
+          m_use = m_new;
+          rescale = (m != -INFINITY);
+          alpha = rescale ? ex2(m - m_new) : 0.f;
+        }
+        const float mu = (m_use == -INFINITY) ? 0.f : m_use;
+        float rsa[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) rsa[a] = 0.f;
+        uint32_t pk[BN / 64][32];
+#pragma unroll
+        for (int i = 0; i < BN; i += 2) {
+          const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
+          const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
+          rsa[(i >> 1) & 7] += p0 + p1;
+          pk[i >> 6][(i >> 1) & 31] = pack_bf16x2(p0, p1);
+        }
+        const float rs = ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+        // P (bf16 pairs) over the first BN/2 columns of this S slot
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) tmem_st32(scol + c * 32, pk[c]);
+        // O must hold P V of every earlier tile of the item before it is
+        // rescaled; that is the only case in which the softmax waits for the
+        // tensor core.  Seeing S(T) implies P V(T-2) is complete (it was
+        // issued before Q K^T(T)), so o_done is at most one phase behind and
+        // its parity wait is exact.
+        if (__any_sync(0xffffffffu, rescale) && j >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, tmo, P.status, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < C::DV / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        l = (rescale ? l * alpha : l) + rs;
+        m = m_use;
+        tc_fence_before();
+        mbar_arrive(&p_full[T & 1]);
+        if (t == 0 && I == 0 && j < 120) mark(128 + j);
+      }
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, I & 1, tmo, P.status, abort_flag));
+      if (ok) {
+        // epilogue: O / l -> bf16, thread t writing row t's DV dims to global
+        // memory; then O is free for the next item
+        if (t == 0 && I == 0) mark(4);
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* orow = reinterpret_cast<uint4*>(
+            P.out + ((static_cast<size_t>(w.b) * S + (valid ? qi : 0)) * H + w.h) * D + w.dv_lo);
 #pragma unroll 1
         for (int c = 0; c < C::DV / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
           tmem_wait_ld();
+          if (valid) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
+            for (int v = 0; v < 4; ++v) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+              u.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+              u.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+              u.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+              orow[4 * c + v] = u;
+            }
+          }
         }
       }
-      tmem_wait_st();
-      l = (rescale ? l * alpha : l) + rs;
-      m = m_use;
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
-      if (t == 0 && j < 120) mark(128 + j);
+      mbar_arrive(o_empty);
+      T0 += w.ntiles;
+      ++I;
     }
-    ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, tmo, P.status, abort_flag));
-    if (ok) {
-      // epilogue: O / l -> bf16 into the (now idle) Q tile area, then TMA store
-      if (t == 0) mark(4);
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint8_t* orow = smem + C::OFF_Q + t * 128;
-#pragma unroll 1
-      for (int c = 0; c < C::DV / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-          const int ch = 4 * c + v;
-          *reinterpret_cast<uint4*>(orow + (ch >> 3) * C::SLAB128 + (((ch & 7) ^ (t & 7)) << 4)) = u;
-        }
-      }
-      fence_proxy_async_smem();
-      named_barrier(1, 128);
-      if (t == 0) {
-#pragma unroll
-        for (int sl = 0; sl < C::DV / 64; ++sl)
-          tma_store_4d(&P.tm_o, smem + C::OFF_Q + sl * C::SLAB128, dv_lo + sl * 64, h, q0, b);
-        bulk_commit();
-        bulk_wait_read_all();
-      }
-    }
-  } else if (warp == 4) {
+  }
+  else if (warp == 4) {
     // ------------------------------------------------------------------ producer
+    // Each key tile (KCH boxes, ring slots [0, KCH)) and each value tile (VCH
+    // boxes, slots [KCH, NSTAGE)) lands under one barrier phase: a phase per
+    // box would cap this thread's copy stream far below the L2 rate.  Per
+    // item: K(0), then Q (once the previous item's last Q K^T is done with the
+    // Q tile), then K(j), V(j-1) in the order the MMA issuer consumes them.
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-#pragma unroll
-      for (int sl = 0; sl < D / 64; ++sl)
-        tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, h, q0, b);
-      // Each key tile (KCH boxes, slots [0, KCH)) and each value tile (VCH
-      // boxes, slots [KCH, NSTAGE)) lands under one barrier phase: a phase
-      // per box would cap this thread's copy stream far below the L2 rate.
-      uint64_t* kf = &full[0];
-      uint64_t* ke = &empty[0];
-      uint64_t* vf = &full[C::KCH];
-      uint64_t* ve = &empty[C::KCH];
-      auto load_k = [&](int j) -> bool {
-        if (!mbar_wait(ke, (j & 1) ^ 1, tmo, P.status, abort_flag)) return false;
+      auto load_k = [&](const Item& w, int T, int j) -> bool {
+        if (!mbar_wait(ke, (T & 1) ^ 1, tmo, P.status, abort_flag)) return false;
         mbar_arrive_expect_tx(kf, C::KCH * C::SLAB_KV);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_4d(smem + C::OFF_RING + c * C::SLAB_KV, &P.tm_k, kf, c * 64, kvh, tile_key(j), b);
+          tma_load_4d(smem + C::OFF_RING + c * C::SLAB_KV, &P.tm_k, kf, c * 64, w.kvh, tile_key(w, j), w.b);
         return true;
       };
-      auto load_v = [&](int j) -> bool {
-        if (!mbar_wait(ve, (j & 1) ^ 1, tmo, P.status, abort_flag)) return false;
+      auto load_v = [&](const Item& w, int T, int j) -> bool {
+        if (!mbar_wait(ve, (T & 1) ^ 1, tmo, P.status, abort_flag)) return false;
         mbar_arrive_expect_tx(vf, C::VCH * C::SLAB_KV);
         for (int c = 0; c < C::VCH; ++c)
-          tma_load_4d(smem + C::OFF_RING + (C::KCH + c) * C::SLAB_KV, &P.tm_v, vf, dv_lo + c * 64, kvh,
-                      tile_key(j), b);
+          tma_load_4d(smem + C::OFF_RING + (C::KCH + c) * C::SLAB_KV, &P.tm_v, vf, w.dv_lo + c * 64, w.kvh,
+                      tile_key(w, j), w.b);
         return true;
       };
-      // same order as the MMA issuer consumes them: K(j) then V(j-1)
       bool ok = true;
-      int lk = -1, lv = -1;  // last key / value tile issued
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = load_k(j);
-        if (ok) lk = j;
-        if (ok && j >= 1) ok = load_v(j - 1);
-        if (ok && j >= 1) lv = j - 1;
+      int T0 = 0, lk = -1, lv = -1, lq = -1;  // last key tile, value tile, Q tile issued
+      for (int r = 0, I = 0; r < nrounds && ok; ++r) {
+      const int it = item_at(r);
+      if (it >= nitems) continue;
+        const Item w = item_of(it);
+        ok = load_k(w, T0, 0);
+        if (!ok) break;
+        lk = T0;
+        ok = mbar_wait(q_empty, (I & 1) ^ 1, tmo, P.status, abort_flag);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+#pragma unroll
+        for (int sl = 0; sl < D / 64; ++sl)
+          tma_load_4d(smem + C::OFF_Q + sl * C::SLAB128, &P.tm_q, q_full, sl * 64, w.h, w.q0, w.b);
+        lq = I;
+        for (int j = 1; j < w.ntiles && ok; ++j) {
+          ok = load_k(w, T0 + j, j);
+          if (ok) lk = T0 + j;
+          if (ok) ok = load_v(w, T0 + j - 1, j - 1);
+          if (ok) lv = T0 + j - 1;
+        }
+        if (ok) ok = load_v(w, T0 + w.ntiles - 1, w.ntiles - 1);
+        if (ok) lv = T0 + w.ntiles - 1;
+        T0 += w.ntiles;
+      ++I;
       }
-      if (ok && load_v(ntiles - 1)) lv = ntiles - 1;
       // let every issued copy land before the CTA can exit
-      mbar_wait(q_full, 0, tmo, P.status, nullptr);
+      if (lq >= 0) mbar_wait(q_full, lq & 1, tmo, P.status, nullptr);
       if (lk >= 0) mbar_wait(kf, lk & 1, tmo, P.status, nullptr);
       if (lv >= 0) mbar_wait(vf, lv & 1, tmo, P.status, nullptr);
     }
-  } else {
+  }
+  else {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::DV, false, true);
-      bool ok = mbar_wait(q_ready, 0, tmo, P.status, abort_flag);
-      mark(3);
-      tc_fence_after();
-      uint64_t* kf = &full[0];
-      uint64_t* ke = &empty[0];
-      uint64_t* vf = &full[C::KCH];
-      uint64_t* ve = &empty[C::KCH];
-      auto qk = [&](int j) -> bool {
-        const uint32_t s_tm = tmem + ((j & 1) ? C::TM_S1 : C::TM_S0);
-        if (!mbar_wait(kf, j & 1, tmo, P.status, abort_flag)) return false;
-        if (j == 0) mark(6);
+      auto qk = [&](int T, bool trace_it, int j) -> bool {
+        const uint32_t s_tm = tmem + ((T & 1) ? C::TM_S1 : C::TM_S0);
+        if (!mbar_wait(kf, T & 1, tmo, P.status, abort_flag)) return false;
+        if (trace_it && j == 0) mark(6);
         tc_fence_after();
         for (int c = 0; c < C::KCH; ++c) {
           const uint32_t kb = sbase + C::OFF_RING + c * C::SLAB_KV;
@@ -395,14 +408,17 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           }
         }
         mma_commit(ke);
-        mma_commit(&s_full[j & 1]);
-        if (j < 120) mark(248 + j);
+        mma_commit(&s_full[T & 1]);
+        if (trace_it && j < 120) mark(248 + j);
         return true;
       };
-      auto pv = [&](int i) -> bool {
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, tmo, P.status, abort_flag)) return false;
-        const uint32_t p_tm = tmem + ((i & 1) ? C::TM_S1 : C::TM_S0);
-        if (!mbar_wait(vf, i & 1, tmo, P.status, abort_flag)) return false;
+      // first: the item's first P V, which overwrites O and so waits until the
+      // softmax has read the previous item's O
+      auto pv = [&](int T, int I, bool first, bool trace_it, int j) -> bool {
+        if (!mbar_wait(&p_full[T & 1], (T >> 1) & 1, tmo, P.status, abort_flag)) return false;
+        if (first && !mbar_wait(o_empty, (I & 1) ^ 1, tmo, P.status, abort_flag)) return false;
+        const uint32_t p_tm = tmem + ((T & 1) ? C::TM_S1 : C::TM_S0);
+        if (!mbar_wait(vf, T & 1, tmo, P.status, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = sbase + C::OFF_RING + C::KCH * C::SLAB_KV;
 #pragma unroll
@@ -410,21 +426,35 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           // 16 keys x 256 value dims, MN-major: key rows 128 B apart, 8-row groups
           // 1 KB apart, 64-dim boxes one slot apart
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, C::SLAB_KV, 1024);
-          mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::TM_O, p_tm + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
         mma_commit(ve);
         mma_commit(o_done);
-        if (i < 120) mark(368 + i);
+        if (trace_it && j < 120) mark(368 + j);
         return true;
       };
-      // issue order Q K^T(j), P V(j-1): the slot of tile j is rewritten by
-      // Q K^T(j+2) only after P V(j), which reads P from it, was issued
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = qk(j);
-        if (ok && j >= 1) ok = pv(j - 1);
+      // issue order Q K^T(T), P V(T-1): the S slot of tile T is rewritten by
+      // Q K^T(T+2) only after P V(T), which reads P from it, was issued
+      bool ok = true;
+      int T0 = 0;
+      for (int r = 0, I = 0; r < nrounds && ok; ++r) {
+      const int it = item_at(r);
+      if (it >= nitems) continue;
+        const Item w = item_of(it);
+        ok = mbar_wait(q_full, I & 1, tmo, P.status, abort_flag);
+        if (!ok) break;
+        if (I == 0) mark(3);
+        tc_fence_after();
+        for (int j = 0; j < w.ntiles && ok; ++j) {
+          ok = qk(T0 + j, I == 0, j);
+          if (ok && j == w.ntiles - 1) mma_commit(q_empty);  // Q is free once this completes
+          if (ok && j >= 1) ok = pv(T0 + j - 1, I, j == 1, I == 0, j - 1);
+        }
+        if (ok) ok = pv(T0 + w.ntiles - 1, I, w.ntiles == 1, I == 0, w.ntiles - 1);
+        mma_commit(o_final);
+        T0 += w.ntiles;
+      ++I;
       }
-      if (ok) pv(ntiles - 1);
-      mma_commit(o_final);
       // every MMA issued above has completed before TMEM is released
       mma_commit(drain);
       mbar_wait(drain, 0, tmo, P.status, nullptr);
@@ -446,11 +476,9 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   PrefillKParams P;
   if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, D, C::BM) ||
       !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN) ||
-      !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN) ||
-      !encode_tmap_bshd(&P.tm_o, pa.out, pa.B, pa.S, la.H, D, C::BM))
+      !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN))
     return cudaErrorInvalidValue;
-  P.positions = pa.positions;
-  P.q_prepared = pa.q_prepared;
+  P.out = pa.out;
   P.status = pa.status;
   P.timeout_ns = pa.timeout_ns;
   P.B = pa.B;
@@ -467,7 +495,14 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const long long grid = static_cast<long long>(P.nqt) * pa.B * la.H * P.dv_splits;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM (the shared memory allows no more), each taking items in turn
+  const long long items = static_cast<long long>(P.nqt) * pa.B * la.H * P.dv_splits;
+  if (items > (1LL << 31) - 1) return cudaErrorInvalidValue;
+  const long long grid = items < sms ? items : sms;
   kern<<<static_cast<unsigned>(grid), 192, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
