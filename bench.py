@@ -255,6 +255,7 @@ def make_decode(wl, dev):
                 metric="decode KV GB/s (algorithmic bytes)", bound="hbm", launches=2,
                 kernel_src=("gemma_family_decoder_b200/csrc/prep_decode.cu",
                             "gemma_family_decoder_b200/csrc/decode_tc.cu",
+                            "gemma_family_decoder_b200/csrc/decode_simt.cu",
                             "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 

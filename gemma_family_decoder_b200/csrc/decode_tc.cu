@@ -510,6 +510,11 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     // the slot it frees.
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NPV, true, false);
+      // Tiles beyond the two shared-memory slots are brought into L2 ahead of
+      // their loads (up to kPrefetch tiles past the one being loaded), so a
+      // slot that frees up refills from L2 instead of waiting on HBM.
+      constexpr int kPrefetch = 4;
+      int pf_next = 2;
       auto load = [&](int j) {
         const int slot = j & 1;
         mbar_arrive_expect_tx(&full[slot], C::RAW);
@@ -517,6 +522,9 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
         for (int c = 0; c < C::NB; ++c)
           tma_load_4d(smem + C::OFF_RAW + slot * C::RAW + c * C::BOX, &P.tm_k, &full[slot], 64 * c,
                       kvh, start + j * C::TK, b);
+        for (; pf_next < ntiles && pf_next <= j + kPrefetch; ++pf_next)
+#pragma unroll
+          for (int c = 0; c < C::NB; ++c) tma_prefetch_l2_4d(&P.tm_k, 64 * c, kvh, start + pf_next * C::TK, b);
         if (j < 24) mark(152 + j);
       };
       int issued = 0;
@@ -637,9 +645,9 @@ static cudaError_t run_decode_tc(const DecodeArgs& da, const LayerArgs& la, cuda
   return cudaGetLastError();
 }
 
-bool decode_tc_supported(const DecodeArgs& da, const LayerArgs& la) {
-  return la.k_eq_v && (la.G == 8 || la.G == 16) && (la.D == 256 || la.D == 512) &&
-         la.rot <= 128 && (reinterpret_cast<uintptr_t>(da.k) & 15) == 0;
+// (The C ABI has already checked that every cache pointer is 16-byte aligned.)
+bool decode_tc_supported(const LayerArgs& la) {
+  return la.k_eq_v && (la.G == 8 || la.G == 16) && (la.D == 256 || la.D == 512) && la.rot <= 128;
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {

@@ -54,13 +54,24 @@ struct DecodeArgs {
   unsigned long long* trace = nullptr;  // optional per-CTA timeline (tensor-core kernel)
   size_t trace_bytes = 0;
 };
-void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk);
+// Split plan of a decode call: keys per chunk and split slots per (b, head),
+// with at most `max_split` slots (fewer, longer chunks when the plan would
+// exceed it; callers check the result against their own limit).
+void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk,
+                 int max_split = 1 << 30);
+// Partials of every split, by the kernel that fits the layer, then nothing else
+// (the merge is launch_decode_combine).
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 // Tensor-core split kernel: K=V layers with 8 or 16 query heads per kv head,
 // head_dim 256 or 512 and at most 128 rotated dims (same partial format).
-bool decode_tc_supported(const DecodeArgs& da, const LayerArgs& la);
+bool decode_tc_supported(const LayerArgs& la);
 cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
+// Persistent CUDA-core split kernel for 1, 2 or 4 query heads per kv head
+// (head_dim 512: 1 or 2) and 1, 2, 4 or 8 kv heads; its own plan.
+bool decode_simt_supported(const LayerArgs& la);
+void decode_simt_plan(const LayerArgs& la, int B, int max_len, int max_split, int* nsplit, int* chunk);
+cudaError_t launch_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 
 // Prefill on tcgen05 tensor cores.
 struct PrefillArgs {

@@ -140,6 +140,15 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Bring one 4-D box into L2 ahead of its load (a hint: no shared memory, no
+// completion to wait for; parts of the box outside the tensor are skipped).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 // 4-D tiled store from shared memory (bulk-group completion).  Rows past the
 // tensor's extent are clipped by the hardware; coordinates are never negative.
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int c0,

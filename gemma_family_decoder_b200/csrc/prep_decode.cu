@@ -326,10 +326,14 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs da, Laye
   }
 }
 
-void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk) {
-  (void)B;
+void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chunk, int max_split) {
+  if (!decode_tc_supported(la) && decode_simt_supported(la)) {
+    decode_simt_plan(la, B, max_len, max_split, nsplit, chunk);
+    return;
+  }
   const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
-  const int c = la.window > 0 ? 256 : 1024;
+  int c = la.window > 0 ? 256 : 1024;
+  if ((span + c - 1) / c > max_split && max_split > 0) c = (span + max_split - 1) / max_split;
   *chunk = c;
   *nsplit = (span + c - 1) / c;
 }
@@ -349,7 +353,8 @@ static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, c
 }
 
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
-  if (decode_tc_supported(da, la)) return launch_decode_tc(da, la, s);
+  if (decode_tc_supported(la)) return launch_decode_tc(da, la, s);
+  if (decode_simt_supported(la)) return launch_decode_simt(da, la, s);
   const int hpw = la.G <= 2 ? la.G : la.G / 4;
   if (la.D == 256) {
     switch (hpw) {
@@ -445,19 +450,15 @@ extern "C" int gattn_decode_noalloc(const gattn_bf16* q, const gattn_bf16* k_cac
   // the normal split plan, with fewer (longer) splits when its partials
   // would not fit the scratch array
   DecodeArgs da;
-  decode_plan(la, batch, max_len, &da.nsplit, &da.chunk);
   const size_t per_split = static_cast<size_t>(batch) * la.H * (la.D + 2) * sizeof(float);
   const size_t usable = kNoAllocScratchBytes - 512;  // room for two 256-byte roundings
-  const int max_split = static_cast<int>(usable / per_split);
-  if (max_split < 1)
+  const size_t fit = usable / per_split;
+  const int max_split = fit > (1u << 30) ? (1 << 30) : static_cast<int>(fit);
+  if (max_split >= 1) decode_plan(la, batch, max_len, &da.nsplit, &da.chunk, max_split);
+  if (max_split < 1 || da.nsplit > max_split)
     return report_error(GATTN_ERR_UNSUPPORTED,
                         "batch * num_heads * (head_dim + 2) * 4 bytes exceed the 16 MiB scratch "
                         "of gattn_decode_noalloc; use gattn_decode with a workspace");
-  if (da.nsplit > max_split) {
-    const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
-    da.chunk = (span + max_split - 1) / max_split;
-    da.nsplit = (span + da.chunk - 1) / da.chunk;
-  }
   void* base = nullptr;
   cudaError_t e = noalloc_scratch_address(&base);
   if (e != cudaSuccess) return report_error(GATTN_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch failed");

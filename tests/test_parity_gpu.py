@@ -180,6 +180,23 @@ DEC_CASES = [
     ("mqa_d256_softcap_norm1", W.Layer(num_heads=8, num_kv_heads=1, head_dim=256, softcap=50.0,
                                        qk_norm=W.NORM_ONE_PLUS_W, window=300), [1, 299, 300, 301, 900]),
     ("gqa4_d256", W.Layer(num_heads=16, num_kv_heads=4, head_dim=256, rope_theta=1e6), [7, 600]),
+    # persistent CUDA-core split kernel (1, 2 or 4 query heads per kv head): every
+    # RoPE branch (none, partner lane R/8 away, one or two same-lane groups),
+    # both norm modes, softcap, window, K=V, head_dim 512, 1/2/4/8 kv heads
+    ("simt_g1_d512_keqv_r128_norm", W.Layer(num_heads=2, num_kv_heads=2, head_dim=512,
+                                            rotary_fraction=0.25, scalar=512.0, k_eq_v=True,
+                                            qk_norm=W.NORM_W), [1, 33, 700]),
+    ("simt_g2_d512_cap_w300_r256", W.Layer(num_heads=4, num_kv_heads=2, head_dim=512, softcap=50.0,
+                                           window=300, rotary_fraction=0.5, scalar=512.0),
+     [5, 299, 300, 301, 1000]),
+    ("simt_g2_d512_full_rope", W.Layer(num_heads=2, num_kv_heads=1, head_dim=512, rope_theta=1e6,
+                                       scalar=512.0), [3, 77, 1030]),
+    ("simt_g4_d256_r64_norm1", W.Layer(num_heads=4, num_kv_heads=1, head_dim=256, rotary_fraction=0.25,
+                                       qk_norm=W.NORM_ONE_PLUS_W), [2, 100, 513]),
+    ("simt_g1_d256_norope_keqv", W.Layer(num_heads=8, num_kv_heads=8, head_dim=256,
+                                         rotary_fraction=0.0, k_eq_v=True), [1, 9, 64, 65]),
+    ("simt_g2_d256_r16_cap_w5", W.Layer(num_heads=8, num_kv_heads=4, head_dim=256, rotary_fraction=0.0625,
+                                        softcap=30.0, window=5), [1, 4, 5, 6, 40]),
     # tensor-core split kernel (K=V, 8 or 16 query heads per kv head, <= 128 rotated dims)
     ("keqv_g8_d512_norm", W.Layer(num_heads=8, num_kv_heads=1, head_dim=512, rope_theta=1e6,
                                   rotary_fraction=0.25, scalar=512.0, k_eq_v=True,
