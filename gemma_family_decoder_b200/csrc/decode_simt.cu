@@ -8,8 +8,9 @@
 //   major, are cut into equal contiguous ranges, one per CTA; the chunks of one
 //   sequence inside a range form a segment, streamed as one key range.
 // * A tile is 32 KB of consecutive cache rows (all kv heads of TP positions),
-//   moved by one bulk copy (and the value rows by a second) into a ring of
-//   stages that a single producer thread keeps full.
+//   moved by one bulk copy (and the value rows by a second, and the rows of
+//   the RoPE table for its positions by a third) into a ring of stages; the
+//   last warp to finish with a stage refills it.
 // * Warp w (of 8) serves kv head w % Hkv and, of every tile, the positions
 //   sub + SUB r (sub = w / Hkv, SUB = 8 / Hkv).  Lane l owns dims 4l + 128c + e
 //   (c < D/128, e < 4), so the two dims of a rotate-half pair sit in one lane
@@ -96,6 +97,36 @@ __device__ __forceinline__ Seg segment(const SimtParams& P, int b, long long i0,
   }
   return s;
 }
+
+// Walks the tiles of a CTA's range in order: segment after segment, TP
+// positions at a time.  `next` yields the sequence, the first cache position
+// and the positions of the following tile, or false past the last one.
+struct TileCursor {
+  int b, b_last, p0, pe, TP;
+  long long i0, i1;
+  __device__ __forceinline__ void init(const SimtParams& P, long long i0_, long long i1_, int tp) {
+    i0 = i0_;
+    i1 = i1_;
+    TP = tp;
+    b = static_cast<int>(i0 / P.nch) - 1;
+    b_last = static_cast<int>((i1 - 1) / P.nch);
+    p0 = pe = 0;
+  }
+  __device__ __forceinline__ bool next(const SimtParams& P, int* tb, int* tp0, int* tn) {
+    while (p0 >= pe) {
+      if (b >= b_last) return false;
+      ++b;
+      const Seg sg = segment(P, b, i0, i1);
+      p0 = sg.ps;
+      pe = sg.pe;
+    }
+    *tb = b;
+    *tp0 = p0;
+    *tn = min(TP, pe - p0);
+    p0 += TP;
+    return true;
+  }
+};
 
 // Sum of v[i] over the 32 lanes for every i < NV.  Step s exchanges across
 // lane bit s: a lane with that bit set keeps the upper half of its entries.
@@ -247,7 +278,7 @@ __device__ __forceinline__ void unpack_lane(const uint8_t* row, int lane, float 
 }  // namespace
 
 template <int D, int G, bool KEQV>
-__global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __grid_constant__ SimtParams P) {
+__global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_constant__ SimtParams P) {
   using C = SimtShape<D, G, KEQV>;
   constexpr int NC = C::NC, RPW = C::RPW, NV = C::NV;
   const DecodeArgs& da = P.da;
@@ -255,13 +286,13 @@ __global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* empty = full + C::NST;
+  int* done_cnt = reinterpret_cast<int*>(full + C::NST);  // [NST] warps done with a stage, cumulative
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kSW);
+      done_cnt[s] = 0;
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -281,38 +312,30 @@ __global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __
   // the (cos, sin) rows of a tile's positions travel with the tile when they fit
   const bool tab_staged = half > 0 && TP * half * static_cast<int>(sizeof(float2)) <= kTabBytes;
 
-  if (warp == kSW) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int t = 0;
-      bool ok = true;
-      for (int b = b_first; b <= b_last && ok; ++b) {
-        const Seg sg = segment(P, b, i0, i1);
-        for (int p0 = sg.ps; p0 < sg.pe; p0 += TP, ++t) {
-          const int st = t % C::NST, n = t / C::NST;
-          if (n > 0 && !mbar_wait(&empty[st], (n - 1) & 1, tmo, da.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int npos = min(TP, sg.pe - p0);
-          const uint32_t bytes = static_cast<uint32_t>(npos * row_elems * sizeof(__nv_bfloat16));
-          const size_t off = (static_cast<size_t>(b) * da.max_len + p0) * row_elems;
-          uint8_t* dst = smem + st * C::STAGE;
-          // table rows past the table's end are not copied; their positions
-          // are flagged and clamped by the compute warps
-          const int trows = tab_staged ? max(0, min(npos, la.rope_max_pos - p0)) : 0;
-          const uint32_t tbytes = static_cast<uint32_t>(trows * half * sizeof(float2));
-          mbar_arrive_expect_tx(&full[st], (KEQV ? bytes : 2 * bytes) + tbytes);
-          bulk_load(dst, da.k + off, bytes, &full[st]);
-          if (!KEQV) bulk_load(dst + kTileBytes, da.v + off, bytes, &full[st]);
-          if (tbytes) bulk_load(dst + C::OFF_TAB, la.rope_tab + static_cast<size_t>(p0) * half, tbytes, &full[st]);
-        }
-      }
-      // every copy issued must land before the CTA may exit
-      for (int u = t - C::NST < 0 ? 0 : t - C::NST; u < t; ++u)
-        mbar_wait(&full[u % C::NST], (u / C::NST) & 1, tmo, da.status, nullptr);
-    }
-    return;
+  // ------------------------------------------------------------ tile copies
+  // Stage st of tile u is refilled with tile u + NST by the last warp to finish
+  // tile u (one arrival counter per stage); warp 0 issues the first NST tiles.
+  // Every warp walks the same cursor, NST tiles ahead of the tile it computes.
+  auto issue = [&](int st, int b, int p0, int npos) {
+    const uint32_t bytes = static_cast<uint32_t>(npos * row_elems * sizeof(__nv_bfloat16));
+    const size_t off = (static_cast<size_t>(b) * da.max_len + p0) * row_elems;
+    // table rows past the table's end are not copied; their positions are
+    // flagged and clamped by the compute loop
+    const int trows = tab_staged ? max(0, min(npos, la.rope_max_pos - p0)) : 0;
+    const uint32_t tbytes = static_cast<uint32_t>(trows * half * sizeof(float2));
+    uint8_t* dst = smem + st * C::STAGE;
+    fence_proxy_async_smem();  // this stage's earlier reads come before the copies' writes
+    mbar_arrive_expect_tx(&full[st], (KEQV ? bytes : 2 * bytes) + tbytes);
+    bulk_load(dst, da.k + off, bytes, &full[st]);
+    if (!KEQV) bulk_load(dst + kTileBytes, da.v + off, bytes, &full[st]);
+    if (tbytes) bulk_load(dst + C::OFF_TAB, la.rope_tab + static_cast<size_t>(p0) * half, tbytes, &full[st]);
+  };
+  TileCursor ahead;
+  ahead.init(P, i0, i1, TP);
+  {
+    int tb, tp0, tn;
+    for (int u = 0; u < C::NST && ahead.next(P, &tb, &tp0, &tn); ++u)
+      if (warp == 0 && lane == 0) issue(u, tb, tp0, tn);
   }
 
   // -------------------------------------------------------------- compute
@@ -419,7 +442,7 @@ __global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __
       // over the RB rows before the next starts (loads, norms, rotation,
       // dots), with no branch inside a step on full tiles, so that the rows'
       // instructions interleave.
-      constexpr int RB = RPW < 4 ? RPW : 4;
+      constexpr int RB = RPW;
       float part[NV], ssr[RPW];
       const bool staged = tab_staged && p0 + TP <= la.rope_max_pos;
 #pragma unroll
@@ -578,7 +601,12 @@ __global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __
           }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      {
+        int tb, tp0, tn;
+        const bool more = ahead.next(P, &tb, &tp0, &tn);  // tile t + NST, if any
+        __threadfence_block();  // this warp's reads of the stage are done
+        if (lane == 0 && (atomicAdd(&done_cnt[st], 1) % kSW) == kSW - 1 && more) issue(st, tb, tp0, tn);
+      }
     }
     if (!ok) break;
     // ---- this segment's partial: l per head over the row bits, then O and (m, l)
@@ -599,6 +627,13 @@ __global__ void __launch_bounds__((kSW + 1) * 32, 1) decode_simt_kernel(const __
         da.part_ml[prow * 2] = m[h];
         da.part_ml[prow * 2 + 1] = lh;
       }
+    }
+  }
+  if (*abort_flag) {
+    // after a failed wait, copies issued just before it may still be landing:
+    // give them ~100 us before the CTA may exit
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000) {
     }
   }
 }
@@ -629,7 +664,7 @@ cudaError_t run_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStrea
   const long long items = static_cast<long long>(da.B) * P.nch;
   if (items <= 0) return cudaSuccess;
   const long long grid = items < sms ? items : sms;
-  kern<<<static_cast<unsigned>(grid), (kSW + 1) * 32, C::SMEM, s>>>(P);
+  kern<<<static_cast<unsigned>(grid), kSW * 32, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -294,32 +294,64 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(DecodeA
   }
 }
 
-// Merge the per-chunk partials of one (b, h) row.
+// Merge the per-chunk partials of one (b, h) row: M = max of the partials'
+// maxima, weights 2^(m_c - M) (0 for empty partials), o = sum_c w_c O_c /
+// sum_c w_c l_c.  The (m, l) pairs are read by all threads at once and reduced
+// through shared memory; only partials with a non-zero weight are read.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs da, LayerArgs la) {
   constexpr int PER = D / 128;
+  extern __shared__ float wsm[];  // [nsplit] weights, then [8] reduction scratch
+  float* red = wsm + da.nsplit;
   const int h = blockIdx.x, b = blockIdx.y;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const size_t base = (static_cast<size_t>(b) * la.H + h) * da.nsplit;
-  float M = -INFINITY;
-  for (int s = 0; s < da.nsplit; ++s) {
-    const float l = da.part_ml[(base + s) * 2 + 1];
-    if (l > 0.f) M = fmaxf(M, da.part_ml[(base + s) * 2]);
+  float mloc = -INFINITY;
+  for (int s = t; s < da.nsplit; s += 128) {
+    const float2 ml = *reinterpret_cast<const float2*>(da.part_ml + (base + s) * 2);
+    if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if (lane == 0) red[warp] = mloc;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float dloc = 0.f;
+  for (int s = t; s < da.nsplit; s += 128) {
+    const float2 ml = *reinterpret_cast<const float2*>(da.part_ml + (base + s) * 2);
+    const float f = ml.y > 0.f ? ex2(ml.x - M) : 0.f;
+    wsm[s] = f;
+    dloc += f * ml.y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dloc += __shfl_xor_sync(0xffffffffu, dloc, o);
+  if (lane == 0) red[4 + warp] = dloc;
+  __syncthreads();
+  const float den = (red[4] + red[5]) + (red[6] + red[7]);
   float num[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) num[e] = 0.f;
-  float den = 0.f;
   for (int s = 0; s < da.nsplit; ++s) {
-    const float l = da.part_ml[(base + s) * 2 + 1];
-    if (!(l > 0.f)) continue;
-    const float f = ex2(da.part_ml[(base + s) * 2] - M);
-    den += f * l;
-    const float* src = da.part_o + (base + s) * D + threadIdx.x * PER;
+    const float f = wsm[s];
+    if (f == 0.f) continue;  // uniform over the block
+    const float* src = da.part_o + (base + s) * D + t * PER;
+    if constexpr (PER == 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      num[0] = fmaf(f, v.x, num[0]);
+      num[1] = fmaf(f, v.y, num[1]);
+    } else {
 #pragma unroll
-    for (int e = 0; e < PER; ++e) num[e] += f * src[e];
+      for (int e = 0; e < PER; e += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src + e);
+        num[e] = fmaf(f, v.x, num[e]);
+        num[e + 1] = fmaf(f, v.y, num[e + 1]);
+        num[e + 2] = fmaf(f, v.z, num[e + 2]);
+        num[e + 3] = fmaf(f, v.w, num[e + 3]);
+      }
+    }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  bf16* dst = da.out + (static_cast<size_t>(b) * la.H + h) * D + threadIdx.x * PER;
+  bf16* dst = da.out + (static_cast<size_t>(b) * la.H + h) * D + t * PER;
 #pragma unroll
   for (int e = 0; e < PER; e += 2) {
     *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(num[e] * inv, num[e + 1] * inv);
@@ -373,10 +405,12 @@ cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaS
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  const size_t smem = (static_cast<size_t>(da.nsplit) + 8) * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
   if (la.D == 256)
-    decode_combine_kernel<256><<<dim3(la.H, da.B), 128, 0, s>>>(da, la);
+    decode_combine_kernel<256><<<dim3(la.H, da.B), 128, smem, s>>>(da, la);
   else
-    decode_combine_kernel<512><<<dim3(la.H, da.B), 128, 0, s>>>(da, la);
+    decode_combine_kernel<512><<<dim3(la.H, da.B), 128, smem, s>>>(da, la);
   return cudaGetLastError();
 }
 
