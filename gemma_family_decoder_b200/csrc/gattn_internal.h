@@ -98,6 +98,24 @@ int check_decode_call(const gattn_cfg* cfg, const void* q, const void* k_cache,
 // Record `msg` as this thread's last error and return `code`.
 int report_error(int code, const char* msg);
 
+// Launch `kern` on `s` with programmatic stream serialization: its CTAs may be
+// scheduled before the previous kernel in the stream finishes, and must call
+// pdl_wait() before reading what that kernel wrote.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Wait limit used by every launch (ns).
 uint64_t wait_timeout_ns();
 

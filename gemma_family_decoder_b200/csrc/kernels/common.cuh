@@ -370,6 +370,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it in the stream is still running; pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op otherwise).  The
+// earlier kernel calls pdl_launch_dependents() to let the later one start.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- small math helpers --------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -175,6 +175,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue kernel's queries and keys are complete and visible past here
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = P.timeout_ns;
   unsigned long long* trace = (P.trace && static_cast<int>(blockIdx.x) < P.trace_ctas)
@@ -503,8 +505,7 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   const long long items = static_cast<long long>(P.nqt) * pa.B * la.H * P.dv_splits;
   if (items > (1LL << 31) - 1) return cudaErrorInvalidValue;
   const long long grid = items < sms ? items : sms;
-  kern<<<static_cast<unsigned>(grid), 192, C::SMEM, s>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(192), C::SMEM, s, P);
 }
 
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {

@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
                                                      bf16* __restrict__ qt, bf16* __restrict__ kt,
                                                      long long tokens, LayerArgs la, uint32_t* status) {
   constexpr int D = TPR * 16;
+  pdl_launch_dependents();  // the attention kernel may be scheduled now; it waits for this grid
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long bs = gid / TPR;
   const int i = static_cast<int>(gid % TPR);
@@ -303,6 +304,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs da, Laye
   constexpr int PER = D / 128;
   extern __shared__ float wsm[];  // [nsplit] weights, then [8] reduction scratch
   float* red = wsm + da.nsplit;
+  pdl_wait();  // the split kernel's partials are complete and visible past here
   const int h = blockIdx.x, b = blockIdx.y;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const size_t base = (static_cast<size_t>(b) * la.H + h) * da.nsplit;
@@ -407,11 +409,8 @@ cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaS
 cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
   const size_t smem = (static_cast<size_t>(da.nsplit) + 8) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  if (la.D == 256)
-    decode_combine_kernel<256><<<dim3(la.H, da.B), 128, smem, s>>>(da, la);
-  else
-    decode_combine_kernel<512><<<dim3(la.H, da.B), 128, smem, s>>>(da, la);
-  return cudaGetLastError();
+  if (la.D == 256) return launch_pdl(decode_combine_kernel<256>, dim3(la.H, da.B), dim3(128), smem, s, da, la);
+  return launch_pdl(decode_combine_kernel<512>, dim3(la.H, da.B), dim3(128), smem, s, da, la);
 }
 
 // ---------------------------------------------------------------------------
