@@ -19,6 +19,7 @@ oracle instead (rank 0 only), on a bounded sample per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -266,6 +267,10 @@ def run_ours(args, world, rank, local):
     name = args.workload
     is_prefill = name in PREFILL_WL
     wl = PREFILL_WL[name] if is_prefill else DECODE_WL[name]
+    if args.len_hi and not is_prefill:
+        # a smaller cache for profiling; with a window no longer than the
+        # shortest sequence the work per step is the same
+        wl = dataclasses.replace(wl, len_hi=max(wl.len_lo, args.len_hi))
     R = make_prefill(wl, dev) if is_prefill else make_decode(wl, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -374,6 +379,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": name, "l2": "flushed before every step (256 MiB write, then a 256 MiB read "
                    "that drains the write's dirty lines), outside the per-step CUDA-event time",
                    "step": "eager library call" if graph is None else "CUDA-graph replay of the library call",
+                   **({"len_hi": wl.len_hi} if args.len_hi and not is_prefill else {}),
                    "parallelism": f"replicas{world}"},
         "roofline": {"bound": R["bound"], "achieved": round(achieved, 3), "peak": peak,
                      "unit": peak_unit, "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -519,6 +525,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(PREFILL_WL) + sorted(DECODE_WL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager library calls instead of a graph replay")
+    ap.add_argument("--len-hi", type=int, default=0,
+                    help="decode: draw sequence lengths up to this (and size the cache for it); for profiling")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     args = ap.parse_args(argv)
     if args.warmup < 3:
