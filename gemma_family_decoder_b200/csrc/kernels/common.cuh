@@ -387,6 +387,30 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^a for two values on the FMA pipe instead of the MUFU unit, for a <= 0 (the
+// exponent of a softmax weight).  a = n + f with n = round(a) and |f| <= 1/2:
+// adding 1.5 * 2^23 leaves n in the low mantissa bits of t; 2^f comes from a
+// cubic fitted here to 2^f on [-1/2, 1/2] (weighted least squares on Chebyshev
+// nodes, reweighted toward the error peaks; relative error < 7.5e-5, far below
+// the bf16 rounding the weights get), and n is added to its exponent field.
+// Arguments below -120 (masked entries are -inf) give exactly 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 a) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.055171653628349304f;
+  const bool zx = a.x < -120.f, zy = a.y < -120.f;
+  a.x = zx ? -120.f : a.x;
+  a.y = zy ? -120.f : a.y;
+  const float2 t = __fadd2_rn(a, make_float2(kRound, kRound));
+  const float2 r = __fadd2_rn(t, make_float2(-kRound, -kRound));  // n, exactly
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), a);     // a - n, exactly
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(zx ? 0.f : __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     zy ? 0.f : __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ float tanh_fast(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -264,8 +264,18 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         uint32_t pk[BN / 64][32];
 #pragma unroll
         for (int i = 0; i < BN; i += 2) {
-          const float p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
-          const float p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
+          // one pair in eight on the FMA pipe: the MUFU unit, 16 exponentials
+          // per clock per SM, is what bounds this loop
+          float p0, p1;
+          if ((i & 15) == 14) {
+            const float2 e = ex2_poly2(CAP ? make_float2(x[i] - mu, x[i + 1] - mu)
+                                           : make_float2(fmaf(x[i], sl2, -mu), fmaf(x[i + 1], sl2, -mu)));
+            p0 = e.x;
+            p1 = e.y;
+          } else {
+            p0 = CAP ? ex2(x[i] - mu) : ex2(fmaf(x[i], sl2, -mu));
+            p1 = CAP ? ex2(x[i + 1] - mu) : ex2(fmaf(x[i + 1], sl2, -mu));
+          }
           rsa[(i >> 1) & 7] += p0 + p1;
           pk[i >> 6][(i >> 1) & 31] = pack_bf16x2(p0, p1);
         }
