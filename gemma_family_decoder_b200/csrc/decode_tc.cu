@@ -2,19 +2,29 @@
 // key/value head (the Gemma 4 global layer: 16 query heads on one K=V head).
 //
 // One CTA takes one chunk of one sequence's cache for one key/value head, in
-// 64-key tiles.  With the keys as the MMA's M dimension ("swap AB"):
-//   S^T [64 keys x G heads] = K~ [64 x D] . Q~^T [D x G]        (M=64, N=G)
-//   O^T [D x G]            += V^T [D x 64] . P^T [64 x G]       (M=128 per 128 dims)
-// K~ is the raw key tile except on the rotated dims [0, R): those are rotated
-// (and given the QK-norm gain) by CUDA cores into a small side tile, and the
-// per-key norm 1/rms(k) is applied to S^T as a scale.  On the unrotated dims the
-// gain is folded into the query instead.  With K=V the values are the raw tile
-// already in shared memory.  The result is the same (m, l, O) partial per
-// (b, head, chunk) as the SIMT split kernel, merged by decode_combine_kernel.
+// 128-key tiles.  With the keys as the MMA's M dimension ("swap AB"):
+//   S^T [128 keys x 16] = K~ [128 x D] . Q~^T [D x 16]       (M=128, N=16)
+//   O^T [D x 16]       += V^T [D x 128] . P^T [128 x 16]     (M=128 per 128 dims)
+// (the group's G heads are the first G of the 16 columns).  A small
+// tcgen05.mma costs a fixed ~46-77 cycles whatever N is, so 128 keys per
+// instruction halve the Q K^T instruction count of 64-key tiles; a 128-key tile
+// of head_dim 512 is 128 KB, too large to keep two of in shared memory for
+// both products, so every tile streams through the shared-memory ring twice:
+// once for Q K^T, its rotated dims rotated in place, and once more (from L2,
+// where the first pass left it) for P V, as raw values.  The ring holds three
+// 64 KB units (four 64-dim boxes of 128 keys); the producer streams Q K^T(j)
+// units, then P V(j-1) units, so tile j's products overlap tile j-1's softmax.
+// K~ is the raw key times the QK-norm gain, rotated, on dims [0, R); on the
+// other dims the gain is folded into the query, and the key norm 1/rms(k) is a
+// per-key scale of S^T.  With K=V the values are the raw tile.  The result is
+// the same (m, l, O) partial per (b, head, chunk) as the other split kernels,
+// merged by decode_combine_kernel.
 //
-// Warps: 0-3 softmax over each tile's S^T (thread = key; TMEM lanes 0-15 of each
-// quadrant hold the 64 rows of an M=64 accumulator) and the epilogue (thread =
-// value dim); 4-7 the key prologue of each tile; 8 TMA producer; 9 MMA issuer.
+// Warps: 0-3 softmax over each tile's S^T (thread = key; TMEM lane = key) and
+// the epilogue (thread = value dim); 4-11 two threads per key: key norms, the
+// in-place rotation, and zeroing of rows past the chunk's end (so that P V
+// multiplies 0 by 0 there, not by stale or poisoned data); 12 TMA producer;
+// 13 MMA issuer.
 #include <cuda_bf16.h>
 
 #include "gattn_internal.h"
@@ -27,37 +37,40 @@ namespace {
 
 template <int D, int G>
 struct DecShape {
-  static constexpr int TK = 64;                  // keys per tile
-  static constexpr int BOX = TK * 128;           // 64 dims x 64 keys
-  static constexpr int NB = D / 64;              // boxes per raw tile
-  static constexpr int RAW = NB * BOX;           // raw key tile
-  static constexpr int NSTAGE = 2;
-  static constexpr int ROT_MAX = 128;            // rotated dims handled by the side tile
-  static constexpr int ROTB = ROT_MAX / 64;      // side-tile boxes
-  static constexpr int QSLAB = G * 128;          // Q^T operand: G head rows x 64 dims
-  static constexpr int NPV = G < 16 ? 16 : G;    // N of P V (M=128 needs N % 16 == 0)
-  static constexpr int PSLAB = NPV * 128;        // P^T: NPV head rows x 64 keys
-  static constexpr int OFF_RAW = 0;
-  static constexpr int OFF_ROT = OFF_RAW + NSTAGE * RAW;
-  static constexpr int OFF_Q = OFF_ROT + NSTAGE * ROTB * BOX;
-  static constexpr int OFF_P = OFF_Q + NB * QSLAB;
-  static constexpr int OFF_RSTEP = OFF_P + NSTAGE * PSLAB;  // (cos, sin) of a 64-position step, [64]
-  static constexpr int OFF_RED = OFF_RSTEP + 64 * 8;        // head maxima [2][4][G], sums [4][G]
-  static constexpr int OFF_BAR = OFF_RED + 3 * 4 * G * 4;
-  static constexpr int NBAR = 16;
+  static constexpr int TK = 128;                 // keys per tile
+  static constexpr int BOX = TK * 128;           // 64 dims x 128 keys
+  static constexpr int NBX = D / 64;             // boxes per tile
+  static constexpr int UB = 4;                   // boxes per ring unit
+  static constexpr int UNIT = UB * BOX;          // 64 KB
+  static constexpr int NCH = NBX / UB;           // units per pass over a tile
+  static constexpr int NSLOT = 3;                // ring units
+  static constexpr int NQ = 16;                  // N of both products (G padded)
+  static constexpr int QSLAB = NQ * 128;         // Q^T operand: 16 head rows x 64 dims
+  static constexpr int PATOM = NQ * 128;         // P^T: 16 head rows x 64 keys
+  static constexpr int PSLAB = 2 * PATOM;        // P^T of a 128-key tile
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_Q = OFF_RING + NSLOT * UNIT;
+  static constexpr int OFF_P = OFF_Q + NBX * QSLAB;
+  static constexpr int OFF_RSTEP = OFF_P + 2 * PSLAB;        // (cos, sin) of a 128-position step, [64]
+  static constexpr int OFF_RN = OFF_RSTEP + 64 * 8;          // key 1/rms, [2][128]
+  static constexpr int OFF_RED = OFF_RN + 2 * TK * 4;        // head maxima [2][4][16], sums [4][16]
+  static constexpr int OFF_BAR = OFF_RED + 3 * 4 * 16 * 4;
+  static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr uint32_t TM_S0 = 0;           // S^T slots: G columns each
-  static constexpr uint32_t TM_S1 = 32;
-  static constexpr uint32_t TM_O = 64;           // O^T: D/128 chunks of NPV columns
+  static constexpr uint32_t TM_S0 = 0;           // S^T slots: 16 columns each
+  static constexpr uint32_t TM_S1 = 16;
+  static constexpr uint32_t TM_O = 32;           // O^T: D/128 blocks of 16 columns
   static constexpr uint32_t TMEM_COLS = 128;
+  static constexpr int THREADS = 14 * 32;
   static_assert(G == 8 || G == 16, "query group of 8 or 16 heads");
-  static_assert(TM_O + (D / 128) * NPV <= TMEM_COLS, "TMEM budget");
+  static_assert(NBX % UB == 0, "whole units");
+  static_assert(TM_O + (D / 128) * NQ <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct DecTcParams {
-  CUtensorMap tm_k;   // cache [B][Lmax][Hkv][D], box 64 dims x 64 keys (keys = values)
+  CUtensorMap tm_k;   // cache [B][Lmax][Hkv][D], box 64 dims x 128 keys (keys = values)
   DecodeArgs da;
   LayerArgs la;
   uint64_t timeout_ns;
@@ -65,10 +78,39 @@ struct DecTcParams {
 
 constexpr float kLog2eD = 1.4426950408889634f;
 
+// Ring unit u of a chunk of n tiles: unit blocks in the order Q K^T(0),
+// Q K^T(1), P V(0), Q K^T(2), P V(1), ..., Q K^T(n-1), P V(n-2), P V(n-1),
+// each NCH units long.
+struct UnitOf {
+  int tile;
+  bool pv;
+  int c;  // unit within the pass
+};
+template <int NCH>
+__device__ __forceinline__ UnitOf unit_of(int u, int n) {
+  const int blk = u / NCH;
+  UnitOf r;
+  r.c = u % NCH;
+  if (blk == 0) {
+    r.tile = 0;
+    r.pv = false;
+  } else if (blk == 2 * n - 1) {
+    r.tile = n - 1;
+    r.pv = true;
+  } else if (blk & 1) {
+    r.tile = (blk + 1) >> 1;
+    r.pv = false;
+  } else {
+    r.tile = (blk >> 1) - 1;
+    r.pv = true;
+  }
+  return r;
+}
+
 }  // namespace
 
 template <int D, int G>
-__global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant__ DecTcParams P) {
+__global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(const __grid_constant__ DecTcParams P) {
   using C = DecShape<D, G>;
   const DecodeArgs& da = P.da;
   const LayerArgs& la = P.la;
@@ -89,43 +131,52 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     return;
   }
   const int ntiles = (end - start + C::TK - 1) / C::TK;
+  const int nunits = 2 * ntiles * C::NCH;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;            // [2] raw tile landed (TMA bytes)
-  uint64_t* raw_empty = bars + 2;   // [2] P V done with the raw tile and P^T slot
-  uint64_t* rot_full = bars + 4;    // [2] key prologue done (128 arrivals)
-  uint64_t* rot_empty = bars + 6;   // [2] Q K^T done with the side tile
-  uint64_t* s_full = bars + 8;      // [2] S^T ready
-  uint64_t* p_full = bars + 10;     // [2] P^T written, O rescaled, S read (128 arrivals)
-  // bars + 12: unused
-  uint64_t* o_final = bars + 13;
-  uint64_t* q_ready = bars + 14;    // 256 arrivals (warps 0-7)
-  uint64_t* drain = bars + 15;
+  uint64_t* full = bars;            // [3] ring unit landed (TMA bytes)
+  uint64_t* ready = bars + 3;       // [3] unit prepared by warps 4-11 (256 arrivals)
+  uint64_t* empty = bars + 6;       // [3] the MMAs are done with the unit
+  uint64_t* s_full = bars + 9;      // [2] S^T of a tile ready
+  uint64_t* p_full = bars + 11;     // [2] P^T written, O rescaled, S read (128 arrivals)
+  uint64_t* p_empty = bars + 13;    // [2] P V done with a P^T slot
+  uint64_t* rn_full = bars + 15;    // [2] key norms of a tile written (256 arrivals)
+  uint64_t* rn_empty = bars + 17;   // [2] the softmax has read them (128 arrivals)
+  uint64_t* o_done = bars + 19;     // one phase per tile's P V
+  uint64_t* o_final = bars + 20;
+  uint64_t* q_ready = bars + 21;    // 256 arrivals (warps 0-7)
+  uint64_t* drain = bars + 22;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);    // [3][4][G]
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);    // [3][4][16]
+  float* rnbuf = reinterpret_cast<float*>(smem + C::OFF_RN);   // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&raw_empty[i], 1);
-      mbar_init(&rot_full[i], 128);
-      mbar_init(&rot_empty[i], 1);
+      mbar_init(&ready[i], 256);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      mbar_init(&p_empty[i], 1);
+      mbar_init(&rn_full[i], 256);
+      mbar_init(&rn_empty[i], 128);
     }
+    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(q_ready, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8 && lane == 0) tma_prefetch_desc(&P.tm_k);
-  if (warp == 9) {
+  if (warp == 12 && lane == 0) tma_prefetch_desc(&P.tm_k);
+  if (warp == 13) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -134,41 +185,25 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = P.timeout_ns;
-  // optional timeline of this CTA (512 entries; layout in the public header)
-  const long long cta = (static_cast<long long>(b) * la.Hkv + kvh) * da.nsplit + split;
-  unsigned long long* trace =
-      (da.trace && cta < static_cast<long long>(da.trace_bytes / (512 * sizeof(unsigned long long))))
-          ? da.trace + cta * 512 : nullptr;
-  const uint64_t t_start = trace ? globaltimer_ns() : 0;
-  auto mark = [&](int slot) {
-    if (trace) trace[slot] = globaltimer_ns() - t_start;
-  };
-  if (trace && threadIdx.x == 0) {
-    uint32_t smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    trace[0] = t_start;
-    trace[1] = smid;
-    trace[2] = ntiles;
-  }
+
   if (warp < 8) {
     // ------------------------------------------------------------ query rows
     // Warps 0-7, one head per warp at a time: QK-norm and RoPE at position L-1
     // into the Q^T operand.  On the unrotated dims the key's gain is applied
-    // here instead of to the keys.  Every row is loaded before any is
-    // transformed, so the global reads overlap.
-    constexpr int NCH = D / 256;
+    // here instead of to the keys.  Rows G..15 of Q^T and P^T stay zero.
+    constexpr int NCHQ = D / 256;
     constexpr int HPW = (G + 7) / 8;
     const float koff = la.qk_norm == 1 ? 1.f : 0.f;
     const float4* gk4 = reinterpret_cast<const float4*>(la.k_norm_w);
-    float x[HPW][NCH][8];
+    float x[HPW][NCHQ][8];
 #pragma unroll
-    for (int hh = 0; hh < HPW; ++hh) load_row<NCH>(da.q + (head0 + warp + 8 * hh) * D, lane, x[hh]);
+    for (int hh = 0; hh < HPW; ++hh) load_row<NCHQ>(da.q + (head0 + warp + 8 * hh) * D, lane, x[hh]);
 #pragma unroll
     for (int hh = 0; hh < HPW; ++hh) {
       const int h = warp + 8 * hh;
-      transform_row<NCH>(x[hh], lane, L - 1, la, la.q_norm_w, da.status);
+      transform_row<NCHQ>(x[hh], lane, L - 1, la, la.q_norm_w, da.status);
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
+      for (int i = 0; i < NCHQ; ++i) {
         const int c = lane + 32 * i;  // 8-dim chunk
         if (la.qk_norm && 8 * c >= la.rot) {
           const float4 g0 = __ldg(gk4 + 2 * c), g1 = __ldg(gk4 + 2 * c + 1);
@@ -181,12 +216,16 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
                                   (((c & 7) ^ (h & 7)) << 4)) = pack8(x[hh][i]);
       }
     }
-    // P^T rows past the group (N padding of P V) stay zero
-    if constexpr (C::NPV > G) {
-      for (int i = threadIdx.x; i < 2 * (C::NPV - G) * 8; i += 256) {
-        const int sl = i / ((C::NPV - G) * 8), r = i % ((C::NPV - G) * 8);
-        *reinterpret_cast<uint4*>(smem + C::OFF_P + sl * C::PSLAB + G * 128 + r * 16) =
-            make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (G < C::NQ) {
+      // zero rows G..15 of every Q^T slab and of both P^T slots
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = threadIdx.x; i < C::NBX * (C::NQ - G) * 8; i += 256) {
+        const int sl = i / ((C::NQ - G) * 8), r = i % ((C::NQ - G) * 8);
+        *reinterpret_cast<uint4*>(smem + C::OFF_Q + sl * C::QSLAB + G * 128 + r * 16) = z;
+      }
+      for (int i = threadIdx.x; i < 4 * (C::NQ - G) * 8; i += 256) {
+        const int at = i / ((C::NQ - G) * 8), r = i % ((C::NQ - G) * 8);
+        *reinterpret_cast<uint4*>(smem + C::OFF_P + at * C::PATOM + G * 128 + r * 16) = z;
       }
     }
     fence_proxy_async_smem();
@@ -194,23 +233,17 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   }
   if (warp < 4) {
     // ------------------------------------------------------------ softmax
-    // Thread (warp w, lane i) serves key kt = 16 w + i%16 of each tile: lanes
-    // i and i+16 sum the squares of its two halves of dims (the key's norm,
-    // taken while the rotation and Q K^T run), and lane i < 16 reads its row
-    // of S^T (TMEM lane 32 w + i holds row 16 w + i of an M=64 accumulator)
-    // with the logits of all G heads.  Maxima are per head over the 64 keys
-    // (warp shuffles, then the 4 warps through shared memory); the running
-    // max m is the same in every thread, so the rescale decision is uniform
-    // over the warpgroup.
+    // Thread t serves key t of each tile: TMEM lane t holds its row of S^T with
+    // the logits of all heads.  Maxima are per head over the tile's 128 keys
+    // (warp shuffles, then the 4 warps through shared memory); the running max
+    // m is the same in every thread, so the rescale decision is uniform.
     const int t = threadIdx.x;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const bool cap = la.softcap > 0.f;
     const float sl2 = la.scale_log2;
     const float kcap = cap ? la.scale / la.softcap : 0.f;
     const float cap_l2 = cap ? la.softcap * kLog2eD : 0.f;
-    const int kt = 16 * warp + (lane & 15);  // key within the tile
-    const int half = lane >> 4;
-    const bool key_lane = lane < 16;
+    const bool odd = lane & 1;
     float m[G], lp[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -221,36 +254,20 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
     for (int j = 0; j < ntiles; ++j) {
       const int slot = j & 1;
       const uint32_t par = (j >> 1) & 1;
-      bool okj = ok && __all_sync(0xffffffffu, mbar_wait(&full[slot], par, tmo, da.status, abort_flag));
+      bool okj = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[slot], par, tmo, da.status, abort_flag));
       float rn = 1.f;
       if (la.qk_norm) {
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        if (okj) {
-          uint8_t* raw = smem + C::OFF_RAW + slot * C::RAW;
-#pragma unroll 4
-          for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c) {
-            float xx[8];
-            unpack8(*tile_chunk(raw, C::BOX, kt, c), xx);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(xx[e], xx[e], acc[e]);
-          }
-        }
-        float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-        rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
+        okj = okj && __all_sync(0xffffffffu, mbar_wait(&rn_full[slot], par, tmo, da.status, abort_flag));
+        rn = rnbuf[slot * C::TK + t];
+        mbar_arrive(&rn_empty[slot]);
       }
-      if (t == 0 && j < 24) mark(176 + j);
-      okj = okj && __all_sync(0xffffffffu, mbar_wait(&s_full[slot], par, tmo, da.status, abort_flag));
-      if (t == 0 && j < 24) mark(80 + j);
       float x[G];
       if (okj) {
         tc_fence_after();
-        uint32_t sr[G];
-        tmem_ldg<G>(tmem + lane_off + (slot ? C::TM_S1 : C::TM_S0), sr);
+        uint32_t sr[C::NQ];
+        tmem_ldg<C::NQ>(tmem + lane_off + (slot ? C::TM_S1 : C::TM_S0), sr);
         tmem_wait_ld();
-        const bool vis = key_lane && (start + j * C::TK + kt) < end;
+        const bool vis = (start + j * C::TK + t) < end;
         const float f = rn * (cap ? kcap : sl2);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -273,22 +290,20 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       for (int h = 0; h < G; ++h) alpha[h] = 1.f;
       bool any = false;
       if (named_barrier_or(1, 128, need)) {
-        float* rw = red + (slot * 4 + warp) * G;
+        float* rw = red + (slot * 4 + warp) * 16;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float v = x[h];
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
           if (lane == 0) rw[h] = v;
         }
         ok = named_barrier_and(1, 128, okj);
         if (!ok) break;
-        const float* rr = red + slot * 4 * G;
+        const float* rr = red + slot * 4 * 16;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float mt = fmaxf(fmaxf(rr[h], rr[G + h]), fmaxf(rr[2 * G + h], rr[3 * G + h]));
+          const float mt = fmaxf(fmaxf(rr[h], rr[16 + h]), fmaxf(rr[32 + h], rr[48 + h]));
           const float mn = fmaxf(m[h], mt);
           if (mn > m[h] + 8.f) {
             alpha[h] = m[h] == -INFINITY ? 0.f : ex2(m[h] - mn);
@@ -297,21 +312,15 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
           }
         }
       }
-      if (t == 0 && j < 24) mark(200 + j);
       // P^T slot reuse: P V(j-2), which read it, must be complete
-      if (j >= 2) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&raw_empty[slot], par ^ 1, tmo, da.status, abort_flag)))
-          ok = false;
-      }
-      if (t == 0 && j < 24) mark(248 + j);
-      // P^T row h is one 128-byte swizzled row: key k at chunk (k/8) ^ (h%8),
-      // half-word k%8.  Lanes 2i and 2i+1 (adjacent keys) swap one value so
-      // that each writes a 32-bit word: the even lane for even heads, the odd
-      // lane for odd heads.
+      if (!__all_sync(0xffffffffu, mbar_wait(&p_empty[slot], par ^ 1, tmo, da.status, abort_flag))) ok = false;
+      // P^T row h: keys in two 64-key atoms, key k of an atom at 16-byte chunk
+      // (k/8) ^ (h%8), half-word k%8.  Lanes 2i and 2i+1 (adjacent keys) swap
+      // one value so that each writes a 32-bit word: the even lane for even
+      // heads, the odd lane for odd heads.
       {
-        uint8_t* pbase = smem + C::OFF_P + slot * C::PSLAB;
-        const int kp = kt & ~1;
-        const bool odd = lane & 1;
+        uint8_t* pbase = smem + C::OFF_P + slot * C::PSLAB + (t >> 6) * C::PATOM;
+        const int kp = t & 62;  // even key of the pair, within the atom
 #pragma unroll
         for (int h = 0; h < G; h += 2) {
           const float p0 = ex2(x[h] - (m[h] == -INFINITY ? 0.f : m[h]));
@@ -319,28 +328,25 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
           lp[h] = lp[h] * alpha[h] + p0;
           lp[h + 1] = lp[h + 1] * alpha[h + 1] + p1;
           const float recv = __shfl_xor_sync(0xffffffffu, odd ? p0 : p1, 1);
-          if (key_lane) {
-            const int hh = h + (odd ? 1 : 0);
-            *reinterpret_cast<uint32_t*>(pbase + hh * 128 + (((kp >> 3) ^ (hh & 7)) << 4) + (kp & 7) * 2) =
-                odd ? pack_bf16x2(recv, p1) : pack_bf16x2(p0, recv);
-          }
+          const int hh = h + (odd ? 1 : 0);
+          *reinterpret_cast<uint32_t*>(pbase + hh * 128 + (((kp >> 3) ^ (hh & 7)) << 4) + (kp & 7) * 2) =
+              odd ? pack_bf16x2(recv, p1) : pack_bf16x2(p0, recv);
         }
       }
-      if (t == 0 && j < 24) mark(224 + j);
-      // O must hold P V of every earlier tile before it is rescaled
+      // O must hold P V of every earlier tile before it is rescaled; seeing
+      // S(j) implies P V(j-2) is complete, so o_done is at most one phase behind
       if (any && j >= 1) {
-        const bool okw = __all_sync(0xffffffffu, mbar_wait(&raw_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, tmo,
-                                                           da.status, abort_flag));
+        const bool okw = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, tmo, da.status, abort_flag));
         if (okw) {
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 128; ++c) {
-            uint32_t o[C::NPV];
-            tmem_ldg<C::NPV>(tmem + lane_off + C::TM_O + c * C::NPV, o);
+            uint32_t o[C::NQ];
+            tmem_ldg<C::NQ>(tmem + lane_off + C::TM_O + c * C::NQ, o);
             tmem_wait_ld();
 #pragma unroll
             for (int h = 0; h < G; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-            tmem_stg<C::NPV>(tmem + lane_off + C::TM_O + c * C::NPV, o);
+            tmem_stg<C::NQ>(tmem + lane_off + C::TM_O + c * C::NQ, o);
           }
           tmem_wait_st();
         } else {
@@ -350,31 +356,26 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[slot]);
-      if (lane == 0 && j < 24) mark((t == 0 ? 104 : 368 + 24 * warp) + j);
     }
     // Epilogue: l summed over the tile's keys and the 4 warps; thread t writes
     // value dim 128 c + t of each head's unnormalised O, lane t < G the (m, l)
     // of head t, in the split kernel's partial format.
-    float* rl = red + 2 * 4 * G;
+    float* rl = red + 2 * 4 * 16;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float v = lp[h];
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      if (lane == 0) rl[warp * G + h] = v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) rl[warp * 16 + h] = v;
     }
     ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, 0, tmo, da.status, abort_flag));
     ok = named_barrier_and(1, 128, ok);
-    if (t == 0) mark(4);
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < D / 128; ++c) {
-        uint32_t o[C::NPV];
-        tmem_ldg<C::NPV>(tmem + lane_off + C::TM_O + c * C::NPV, o);
+        uint32_t o[C::NQ];
+        tmem_ldg<C::NQ>(tmem + lane_off + C::TM_O + c * C::NQ, o);
         tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < G; ++h)
@@ -386,34 +387,35 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       if (t == h) {
         float* ml = da.part_ml + ((head0 + h) * da.nsplit + split) * 2;
         ml[0] = ok ? m[h] : -INFINITY;
-        ml[1] = ok ? (rl[h] + rl[G + h]) + (rl[2 * G + h] + rl[3 * G + h]) : 0.f;
+        ml[1] = ok ? (rl[h] + rl[16 + h]) + (rl[32 + h] + rl[48 + h]) : 0.f;
       }
     }
   }
-  else if (warp < 8) {
-    // ------------------------------------------------------------ key prologue
-    // Two threads per key (t4 = 2 k + hf) write the rotated dims [0, R) of
-    // k * gain into the side tile, and zero rows for keys past the chunk's end
-    // so that P V multiplies 0 by 0 there, not by stale data.  Each thread
-    // keeps (cos, sin) of its pairs' angles at its key's position: computed
-    // exactly (pair t turns theta^(-2t/F) / 2pi per position, a geometric
-    // sequence in double precision, reduced mod 1) every 32 tiles, and in
-    // between advanced by the 64-position step of each pair.
-    const int t4 = threadIdx.x - 128;
-    const int k = t4 >> 1, hf = t4 & 1;
+  else if (warp < 12) {
+    // ------------------------------------------------------- key preparation
+    // Two threads per key (t8 = 2 k + hf) prepare each ring unit before the
+    // MMAs read it.  Q K^T units: the key's sum of squares (QK-norm) over the
+    // 16-byte chunks of its parity, and, in the first unit of a tile, the
+    // rotated dims [0, R) of k * gain rotated in place.  P V units of a tile
+    // that ends inside the chunk: rows past the end zeroed.  (cos, sin) of the
+    // thread's pairs at its key's position: computed exactly (pair t turns
+    // theta^(-2t/F) / 2pi per position, a geometric sequence in double
+    // precision, reduced mod 1) every 32 tiles, and in between advanced by the
+    // 128-position step of each pair.
+    const int t8 = threadIdx.x - 128;
+    const int k = t8 >> 1, hf = t8 & 1;
     const int R = la.rot;
-    const int h8 = R >> 4;                  // 8-dim chunks in half the rotated slice (<= 8)
-    const int rch = ((R + 63) >> 6) << 3;   // chunks covered by the side tile's boxes
+    const int h8 = R >> 4;  // 8-dim chunks in half the rotated slice (<= 8)
     const float koff = la.qk_norm == 1 ? 1.f : 0.f;
     const float4* gk4 = reinterpret_cast<const float4*>(la.k_norm_w);
     float2* rstep = reinterpret_cast<float2*>(smem + C::OFF_RSTEP);
     constexpr double kTurnsPerRad = 0.15915494309189533576888376337251;
-    if (t4 < (R >> 1)) {
+    if (t8 < (R >> 1)) {
       double f = kTurnsPerRad;
-      for (int i = 0; i < t4; ++i) f *= la.rope_ratio;
-      rstep[t4] = rope_cos_sin(C::TK, f);
+      for (int i = 0; i < t8; ++i) f *= la.rope_ratio;
+      rstep[t8] = rope_cos_sin(C::TK, f);
     }
-    named_barrier(2, 128);
+    named_barrier(2, 256);
     float2 cs[4][8];
     auto anchor = [&](int pos) {
       double qp[8];
@@ -438,44 +440,61 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
       x[0] *= g0.x + koff; x[1] *= g0.y + koff; x[2] *= g0.z + koff; x[3] *= g0.w + koff;
       x[4] *= g1.x + koff; x[5] *= g1.y + koff; x[6] *= g1.z + koff; x[7] *= g1.w + koff;
     };
-    for (int j = 0; j < ntiles; ++j) {
-      const int slot = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[slot], par, tmo, da.status, abort_flag) &&
-                                       mbar_wait(&rot_empty[slot], par ^ 1, tmo, da.status, abort_flag)))
-        break;
-      if (t4 == 0 && j < 24) mark(8 + j);
-      uint8_t* raw = smem + C::OFF_RAW + slot * C::RAW;
-      uint8_t* rot = smem + C::OFF_ROT + slot * C::ROTB * C::BOX;
-      const int key = start + j * C::TK + k;
-      if (R > 0) {
-        if ((j & 31) == 0) {
-          anchor(checked_pos(min(key, end - 1), la, da.status));
-        } else {
+    float ss = 0.f;
+    // the 256 threads leave the loop together, at a unit's first barrier, or
+    // not at all (a failed wait is carried to the next unit in `okc`)
+    bool okc = true;
+    for (int u = 0; u < nunits; ++u) {
+      const UnitOf uo = unit_of<C::NCH>(u, ntiles);
+      const int slot = u % C::NSLOT;
+      bool okw = okc && __all_sync(0xffffffffu, mbar_wait(&full[slot], (u / C::NSLOT) & 1, tmo, da.status,
+                                                          abort_flag));
+      if (!named_barrier_and(2, 256, okw)) break;
+      uint8_t* ub = smem + C::OFF_RING + slot * C::UNIT;
+      const int key0 = start + uo.tile * C::TK;
+      const int nvalid = min(C::TK, end - key0);
+      if (!uo.pv) {
+        if (la.qk_norm) {
+          float acc[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = hf + 2 * i;
-            if (c < h8) {
+          for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+          for (int c = hf; c < 4 * 8; c += 2) {
+            float xx[8];
+            unpack8(*tile_chunk(ub, C::BOX, k, c), xx);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float2 st = rstep[8 * c + e];
-                const float2 a = cs[i][e];
-                cs[i][e] = make_float2(a.x * st.x - a.y * st.y, a.y * st.x + a.x * st.y);
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(xx[e], xx[e], acc[e]);
+          }
+          ss += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        }
+        if (uo.c == 0 && R > 0) {
+          if (la.qk_norm) named_barrier(2, 256);  // every raw value is read before any is rotated
+          const int key = key0 + k;
+          if ((uo.tile & 31) == 0) {
+            anchor(checked_pos(min(key, end - 1), la, da.status));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int c = hf + 2 * i;
+              if (c < h8) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float2 st = rstep[8 * c + e];
+                  const float2 a = cs[i][e];
+                  cs[i][e] = make_float2(a.x * st.x - a.y * st.y, a.y * st.x + a.x * st.y);
+                }
               }
             }
           }
-        }
-      }
-      if (t4 == 0 && j < 24) mark(296 + j);
-      if (key < end) {
-        if (R > 0) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int c = hf + 2 * i;
             if (c < h8) {
+              uint4* px = tile_chunk(ub, C::BOX, k, c);
+              uint4* py = tile_chunk(ub, C::BOX, k, c + h8);
               float x[8], y[8];
-              unpack8(*tile_chunk(raw, C::BOX, k, c), x);
-              unpack8(*tile_chunk(raw, C::BOX, k, c + h8), y);
+              unpack8(*px, x);
+              unpack8(*py, y);
               gain8(c, x);
               gain8(c + h8, y);
               float xo[8], yo[8];
@@ -484,133 +503,113 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
                 xo[e] = x[e] * cs[i][e].x - y[e] * cs[i][e].y;
                 yo[e] = y[e] * cs[i][e].x + x[e] * cs[i][e].y;
               }
-              *tile_chunk(rot, C::BOX, k, c) = pack8(xo);
-              *tile_chunk(rot, C::BOX, k, c + h8) = pack8(yo);
+              *px = pack8(xo);
+              *py = pack8(yo);
             }
           }
-          // unrotated dims that share a box with rotated ones: copied raw
-          for (int c = 2 * h8 + hf; c < rch; c += 2) *tile_chunk(rot, C::BOX, k, c) = *tile_chunk(raw, C::BOX, k, c);
         }
-      } else {
+        if (uo.c == C::NCH - 1 && la.qk_norm) {
+          // the key's norm: both threads' sums; the softmax reads it per tile
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          const float rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
+          ss = 0.f;
+          const int ts = uo.tile & 1;
+          okc = __all_sync(0xffffffffu, mbar_wait(&rn_empty[ts], ((uo.tile >> 1) & 1) ^ 1, tmo, da.status,
+                                                  abort_flag));
+          if (okc && hf == 0) rnbuf[ts * C::TK + k] = rn;
+          mbar_arrive(&rn_full[ts]);
+        }
+      } else if (k >= nvalid) {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int c = hf; c < D / 8; c += 2) *tile_chunk(raw, C::BOX, k, c) = z;
-        for (int c = hf; c < rch; c += 2) *tile_chunk(rot, C::BOX, k, c) = z;
+#pragma unroll 4
+        for (int c = hf; c < 4 * 8; c += 2) *tile_chunk(ub, C::BOX, k, c) = z;
       }
       fence_proxy_async_smem();
-      mbar_arrive(&rot_full[slot]);
-      if ((t4 & 31) == 0 && j < 24) mark((t4 == 0 ? 32 : 296 + t4 * 3 / 4) + j);
+      mbar_arrive(&ready[slot]);
     }
   }
-  else if (warp == 8) {
-    // ------------------------------------------------- TMA producer, P V issuer
-    // One thread loads tiles 0 and 1, then per tile j issues
-    // O^T += V^T P^T once the softmax has written P^T(j): A = value boxes
-    // (MN-major, M=128 dims over two 64-dim boxes LBO apart), B = P^T
-    // (K-major, N=NPV); and once that P V has completed, loads tile j+2 into
-    // the slot it frees.
+  else if (warp == 12) {
+    // ------------------------------------------------------------- producer
+    // One thread streams the ring units in the MMA issuer's order: each unit
+    // (four 64-dim boxes of the tile's 128 keys) under one barrier phase,
+    // once the MMAs are done with what the slot held.
     if (lane == 0) {
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NPV, true, false);
-      // Tiles beyond the two shared-memory slots are brought into L2 ahead of
-      // their loads (up to kPrefetch tiles past the one being loaded), so a
-      // slot that frees up refills from L2 instead of waiting on HBM.
-      constexpr int kPrefetch = 4;
-      int pf_next = 2;
-      auto load = [&](int j) {
-        const int slot = j & 1;
-        mbar_arrive_expect_tx(&full[slot], C::RAW);
-#pragma unroll
-        for (int c = 0; c < C::NB; ++c)
-          tma_load_4d(smem + C::OFF_RAW + slot * C::RAW + c * C::BOX, &P.tm_k, &full[slot], 64 * c,
-                      kvh, start + j * C::TK, b);
-        for (; pf_next < ntiles && pf_next <= j + kPrefetch; ++pf_next)
-#pragma unroll
-          for (int c = 0; c < C::NB; ++c) tma_prefetch_l2_4d(&P.tm_k, 64 * c, kvh, start + pf_next * C::TK, b);
-        if (j < 24) mark(152 + j);
-      };
       int issued = 0;
-      for (; issued < 2 && issued < ntiles; ++issued) load(issued);
-      bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int slot = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        ok = mbar_wait(&p_full[slot], par, tmo, da.status, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t rawb = sbase + C::OFF_RAW + slot * C::RAW;
-        const uint32_t pb = sbase + C::OFF_P + slot * C::PSLAB;
+      for (int u = 0; u < nunits; ++u) {
+        const UnitOf uo = unit_of<C::NCH>(u, ntiles);
+        const int slot = u % C::NSLOT;
+        if (!mbar_wait(&empty[slot], ((u / C::NSLOT) & 1) ^ 1, tmo, da.status, abort_flag)) break;
+        uint8_t* ub = smem + C::OFF_RING + slot * C::UNIT;
+        mbar_arrive_expect_tx(&full[slot], C::UNIT);
 #pragma unroll
-        for (int mc = 0; mc < D / 128; ++mc)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + C::TM_O + mc * C::NPV,
-                        smem_desc_sw128(rawb + 2 * mc * C::BOX + kk * 2048, C::BOX, 1024),
-                        smem_desc_sw128(pb + kk * 32, 16, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&raw_empty[slot]);
-        if (j < 24) mark(128 + j);
-        if (j + 2 < ntiles) {
-          ok = mbar_wait(&raw_empty[slot], par, tmo, da.status, abort_flag);
-          if (!ok) break;
-          load(j + 2);
-          issued = j + 3;
-        }
+        for (int bx = 0; bx < C::UB; ++bx)
+          tma_load_4d(ub + bx * C::BOX, &P.tm_k, &full[slot], (uo.c * C::UB + bx) * 64, kvh,
+                      start + uo.tile * C::TK, b);
+        issued = u + 1;
       }
-      // o_final completes once every P V above has; the TMEM they write
-      // stays allocated until then
-      mma_commit(o_final);
-      mbar_wait(o_final, 0, tmo, da.status, nullptr);
       // let every issued copy land before the CTA can exit
-      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-        mbar_wait(&full[j & 1], (j >> 1) & 1, tmo, da.status, nullptr);
+      for (int u = issued - C::NSLOT < 0 ? 0 : issued - C::NSLOT; u < issued; ++u)
+        mbar_wait(&full[u % C::NSLOT], (u / C::NSLOT) & 1, tmo, da.status, nullptr);
     }
   }
   else {
     // ------------------------------------------------------------ MMA issuer
-    // S^T = K~ Q~^T: A = key box (K-major, M=64; the side tile's boxes on the
-    // rotated dims), B = Q^T slab (K-major, N=G).  Q K^T(j) waits for its
-    // tile, its side tile, and for the softmax to be done with S(j-2), whose
-    // TMEM slot it rewrites.
+    // Q K^T units: S^T(j) += K~ box . Q~^T box (A = key box, K-major, M=128;
+    // B = Q^T slab, K-major, N=16); the first unit of tile j waits until the
+    // softmax is done with S(j-2), whose TMEM slot it rewrites.  P V units:
+    // O^T += V^T . P^T (A = two value boxes, MN-major, M=128 dims; B = P^T,
+    // K-major, N=16); the first unit of tile j waits for P^T(j).
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(64, G, false, false);
-      const int rotb = (la.rot + 63) >> 6;
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::NQ, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NQ, true, false);
       bool ok = mbar_wait(q_ready, 0, tmo, da.status, abort_flag);
-      mark(3);
-      // The unrotated dims go first, as soon as the tile has landed; the
-      // rotated ones (from the side tile) once the key prologue is done.
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int slot = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        ok = mbar_wait(&full[slot], par, tmo, da.status, abort_flag) &&
-             (j < 2 || mbar_wait(&p_full[slot], par ^ 1, tmo, da.status, abort_flag));
+      for (int u = 0; u < nunits && ok; ++u) {
+        const UnitOf uo = unit_of<C::NCH>(u, ntiles);
+        const int slot = u % C::NSLOT;
+        const int ts = uo.tile & 1;
+        const uint32_t tpar = (uo.tile >> 1) & 1;
+        if (uo.c == 0)
+          ok = uo.pv ? mbar_wait(&p_full[ts], tpar, tmo, da.status, abort_flag)
+                     : mbar_wait(&p_full[ts], tpar ^ 1, tmo, da.status, abort_flag);
+        ok = ok && mbar_wait(&ready[slot], (u / C::NSLOT) & 1, tmo, da.status, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t s_tm = tmem + (slot ? C::TM_S1 : C::TM_S0);
-        const uint32_t rawb = sbase + C::OFF_RAW + slot * C::RAW;
-        const uint32_t rotbase = sbase + C::OFF_ROT + slot * C::ROTB * C::BOX;
-        for (int c = rotb; c < C::NB; ++c) {
-          const uint32_t ab = rawb + c * C::BOX;
-          const uint32_t qb = sbase + C::OFF_Q + c * C::QSLAB;
+        const uint32_t ub = sbase + C::OFF_RING + slot * C::UNIT;
+        if (!uo.pv) {
+          const uint32_t s_tm = tmem + (ts ? C::TM_S1 : C::TM_S0);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(s_tm, smem_desc_sw128(ab + kk * 32, 16, 1024),
-                        smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk, (c > rotb || kk > 0) ? 1u : 0u);
-        }
-        if (j < 24) mark(56 + j);
-        ok = mbar_wait(&rot_full[slot], par, tmo, da.status, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        for (int c = 0; c < rotb; ++c) {
-          const uint32_t ab = rotbase + c * C::BOX;
-          const uint32_t qb = sbase + C::OFF_Q + c * C::QSLAB;
+          for (int bx = 0; bx < C::UB; ++bx) {
+            const uint32_t qb = sbase + C::OFF_Q + (uo.c * C::UB + bx) * C::QSLAB;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(s_tm, smem_desc_sw128(ab + kk * 32, 16, 1024),
-                        smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk,
-                        (rotb < C::NB || c > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(s_tm, smem_desc_sw128(ub + bx * C::BOX + kk * 32, 16, 1024),
+                          smem_desc_sw128(qb + kk * 32, 16, 1024), idesc_qk,
+                          (uo.c > 0 || bx > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[slot]);
+          if (uo.c == C::NCH - 1) mma_commit(&s_full[ts]);
+        } else {
+          const uint32_t pb = sbase + C::OFF_P + ts * C::PSLAB;
+#pragma unroll
+          for (int mbl = 0; mbl < 2; ++mbl) {
+            const int mb = 2 * uo.c + mbl;  // 128-dim block of O^T
+#pragma unroll
+            for (int kk = 0; kk < C::TK / 16; ++kk)
+              mma_bf16_ss(tmem + C::TM_O + mb * C::NQ,
+                          smem_desc_sw128(ub + 2 * mbl * C::BOX + kk * 16 * 128, C::BOX, 1024),
+                          smem_desc_sw128(pb + (kk >> 2) * C::PATOM + (kk & 3) * 32, 16, 1024), idesc_pv,
+                          (uo.tile > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[slot]);
+          if (uo.c == C::NCH - 1) {
+            mma_commit(&p_empty[ts]);
+            mma_commit(o_done);
+          }
         }
-        mma_commit(&rot_empty[slot]);
-        mma_commit(&s_full[slot]);
       }
-      // every MMA issued above has completed before TMEM is released
+      // o_final completes once every product above has; the TMEM they write
+      // stays allocated until then
+      mma_commit(o_final);
       mma_commit(drain);
       mbar_wait(drain, 0, tmo, da.status, nullptr);
     }
@@ -618,11 +617,10 @@ __global__ void __launch_bounds__(320, 1) decode_tc_kernel(const __grid_constant
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-  if (threadIdx.x == 0) mark(5);
 }
 
 template <int D, int G>
@@ -635,13 +633,18 @@ static cudaError_t run_decode_tc(const DecodeArgs& da, const LayerArgs& la, cuda
   P.la = la;
   P.timeout_ns = wait_timeout_ns();
   auto kern = decode_tc_kernel<D, G>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev] = true;
   }
-  kern<<<dim3(da.nsplit, la.Hkv, da.B), 320, C::SMEM, s>>>(P);
+  kern<<<dim3(da.nsplit, la.Hkv, da.B), C::THREADS, C::SMEM, s>>>(P);
   return cudaGetLastError();
 }
 
