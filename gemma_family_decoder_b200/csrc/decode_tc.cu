@@ -84,7 +84,8 @@ constexpr float kLog2eD = 1.4426950408889634f;
 struct UnitOf {
   int tile;
   bool pv;
-  int c;  // unit within the pass
+  int c;    // unit within the pass
+  int db;   // 256-dim block it holds (the rotated dims are in block 0, first)
 };
 template <int NCH>
 __device__ __forceinline__ UnitOf unit_of(int u, int n) {
@@ -104,6 +105,7 @@ __device__ __forceinline__ UnitOf unit_of(int u, int n) {
     r.tile = (blk >> 1) - 1;
     r.pv = true;
   }
+  r.db = r.c;
   return r;
 }
 
@@ -463,29 +465,20 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
             float xx[8];
             unpack8(*tile_chunk(ub, C::BOX, k, c), xx);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(xx[e], xx[e], acc[e]);
+            for (int e = 0; e < 8; e += 2) {
+              const float2 v = make_float2(xx[e], xx[e + 1]);
+              const float2 r2 = __ffma2_rn(v, v, make_float2(acc[e], acc[e + 1]));
+              acc[e] = r2.x;
+              acc[e + 1] = r2.y;
+            }
           }
           ss += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         }
-        if (uo.c == 0 && R > 0) {
+        if (uo.db == 0 && R > 0) {
           if (la.qk_norm) named_barrier(2, 256);  // every raw value is read before any is rotated
-          const int key = key0 + k;
-          if ((uo.tile & 31) == 0) {
-            anchor(checked_pos(min(key, end - 1), la, da.status));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int c = hf + 2 * i;
-              if (c < h8) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const float2 st = rstep[8 * c + e];
-                  const float2 a = cs[i][e];
-                  cs[i][e] = make_float2(a.x * st.x - a.y * st.y, a.y * st.x + a.x * st.y);
-                }
-              }
-            }
-          }
+          // the angles at this tile's positions: exact every 32 tiles, else
+          // advanced (after the previous tile's rotation) by one step
+          if ((uo.tile & 31) == 0) anchor(checked_pos(min(key0 + k, end - 1), la, da.status));
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int c = hf + 2 * i;
@@ -497,14 +490,40 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
               unpack8(*py, y);
               gain8(c, x);
               gain8(c + h8, y);
-              float xo[8], yo[8];
+              // two pairs per packed fp32x2 instruction
+              uint32_t xo[4], yo[4];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                xo[e] = x[e] * cs[i][e].x - y[e] * cs[i][e].y;
-                yo[e] = y[e] * cs[i][e].x + x[e] * cs[i][e].y;
+              for (int e = 0; e < 8; e += 2) {
+                const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
+                const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
+                const float2 x2 = make_float2(x[e], x[e + 1]), y2 = make_float2(y[e], y[e + 1]);
+                const float2 a = __ffma2_rn(x2, co, __fmul2_rn(y2, make_float2(-si.x, -si.y)));
+                const float2 bb = __ffma2_rn(y2, co, __fmul2_rn(x2, si));
+                xo[e >> 1] = pack_bf16x2(a.x, a.y);
+                yo[e >> 1] = pack_bf16x2(bb.x, bb.y);
               }
-              *px = pack8(xo);
-              *py = pack8(yo);
+              *px = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+              *py = make_uint4(yo[0], yo[1], yo[2], yo[3]);
+            }
+          }
+          if (((uo.tile + 1) & 31) != 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int c = hf + 2 * i;
+              if (c < h8) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  // (cos, sin) of two pairs advanced by their steps, packed
+                  const float4 st = *reinterpret_cast<const float4*>(rstep + 8 * c + e);
+                  const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
+                  const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
+                  const float2 sc = make_float2(st.x, st.z), ss2 = make_float2(st.y, st.w);
+                  const float2 nc = __ffma2_rn(co, sc, __fmul2_rn(si, make_float2(-ss2.x, -ss2.y)));
+                  const float2 ns = __ffma2_rn(si, sc, __fmul2_rn(co, ss2));
+                  cs[i][e] = make_float2(nc.x, ns.x);
+                  cs[i][e + 1] = make_float2(nc.y, ns.y);
+                }
+              }
             }
           }
         }
@@ -543,7 +562,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
         mbar_arrive_expect_tx(&full[slot], C::UNIT);
 #pragma unroll
         for (int bx = 0; bx < C::UB; ++bx)
-          tma_load_4d(ub + bx * C::BOX, &P.tm_k, &full[slot], (uo.c * C::UB + bx) * 64, kvh,
+          tma_load_4d(ub + bx * C::BOX, &P.tm_k, &full[slot], (uo.db * C::UB + bx) * 64, kvh,
                       start + uo.tile * C::TK, b);
         issued = u + 1;
       }
@@ -579,7 +598,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           const uint32_t s_tm = tmem + (ts ? C::TM_S1 : C::TM_S0);
 #pragma unroll
           for (int bx = 0; bx < C::UB; ++bx) {
-            const uint32_t qb = sbase + C::OFF_Q + (uo.c * C::UB + bx) * C::QSLAB;
+            const uint32_t qb = sbase + C::OFF_Q + (uo.db * C::UB + bx) * C::QSLAB;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ss(s_tm, smem_desc_sw128(ub + bx * C::BOX + kk * 32, 16, 1024),
@@ -592,7 +611,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           const uint32_t pb = sbase + C::OFF_P + ts * C::PSLAB;
 #pragma unroll
           for (int mbl = 0; mbl < 2; ++mbl) {
-            const int mb = 2 * uo.c + mbl;  // 128-dim block of O^T
+            const int mb = 2 * uo.db + mbl;  // 128-dim block of O^T
 #pragma unroll
             for (int kk = 0; kk < C::TK / 16; ++kk)
               mma_bf16_ss(tmem + C::TM_O + mb * C::NQ,

@@ -366,7 +366,7 @@ void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chun
     return;
   }
   const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
-  int c = la.window > 0 ? 256 : 1024;
+  int c = la.window > 0 ? 256 : 2048;
   if ((span + c - 1) / c > max_split && max_split > 0) c = (span + max_split - 1) / max_split;
   *chunk = c;
   *nsplit = (span + c - 1) / c;
