@@ -479,50 +479,56 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           // the angles at this tile's positions: exact every 32 tiles, else
           // advanced (after the previous tile's rotation) by one step
           if ((uo.tile & 31) == 0) anchor(checked_pos(min(key0 + k, end - 1), la, da.status));
+          // all four chunk pairs loaded first, then rotated, so that their
+          // latencies overlap; pairs past the rotated slice are not stored
+          // (their chunks are still inside the unit's first two boxes)
+          uint4 ux[4], uy[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int c = hf + 2 * i;
-            if (c < h8) {
-              uint4* px = tile_chunk(ub, C::BOX, k, c);
-              uint4* py = tile_chunk(ub, C::BOX, k, c + h8);
-              float x[8], y[8];
-              unpack8(*px, x);
-              unpack8(*py, y);
-              gain8(c, x);
-              gain8(c + h8, y);
-              // two pairs per packed fp32x2 instruction
-              uint32_t xo[4], yo[4];
+            ux[i] = *tile_chunk(ub, C::BOX, k, c);
+            uy[i] = *tile_chunk(ub, C::BOX, k, c + h8);
+          }
 #pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
-                const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
-                const float2 x2 = make_float2(x[e], x[e + 1]), y2 = make_float2(y[e], y[e + 1]);
-                const float2 a = __ffma2_rn(x2, co, __fmul2_rn(y2, make_float2(-si.x, -si.y)));
-                const float2 bb = __ffma2_rn(y2, co, __fmul2_rn(x2, si));
-                xo[e >> 1] = pack_bf16x2(a.x, a.y);
-                yo[e >> 1] = pack_bf16x2(bb.x, bb.y);
-              }
-              *px = make_uint4(xo[0], xo[1], xo[2], xo[3]);
-              *py = make_uint4(yo[0], yo[1], yo[2], yo[3]);
+          for (int i = 0; i < 4; ++i) {
+            const int c = hf + 2 * i;
+            float x[8], y[8];
+            unpack8(ux[i], x);
+            unpack8(uy[i], y);
+            gain8(c, x);
+            gain8(c + h8, y);
+            // two pairs per packed fp32x2 instruction
+            uint32_t xo[4], yo[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
+              const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
+              const float2 x2 = make_float2(x[e], x[e + 1]), y2 = make_float2(y[e], y[e + 1]);
+              const float2 a = __ffma2_rn(x2, co, __fmul2_rn(y2, make_float2(-si.x, -si.y)));
+              const float2 bb = __ffma2_rn(y2, co, __fmul2_rn(x2, si));
+              xo[e >> 1] = pack_bf16x2(a.x, a.y);
+              yo[e >> 1] = pack_bf16x2(bb.x, bb.y);
+            }
+            if (c < h8) {
+              *tile_chunk(ub, C::BOX, k, c) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+              *tile_chunk(ub, C::BOX, k, c + h8) = make_uint4(yo[0], yo[1], yo[2], yo[3]);
             }
           }
           if (((uo.tile + 1) & 31) != 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int c = hf + 2 * i;
-              if (c < h8) {
+              const int c = min(hf + 2 * i, 7);
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                  // (cos, sin) of two pairs advanced by their steps, packed
-                  const float4 st = *reinterpret_cast<const float4*>(rstep + 8 * c + e);
-                  const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
-                  const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
-                  const float2 sc = make_float2(st.x, st.z), ss2 = make_float2(st.y, st.w);
-                  const float2 nc = __ffma2_rn(co, sc, __fmul2_rn(si, make_float2(-ss2.x, -ss2.y)));
-                  const float2 ns = __ffma2_rn(si, sc, __fmul2_rn(co, ss2));
-                  cs[i][e] = make_float2(nc.x, ns.x);
-                  cs[i][e + 1] = make_float2(nc.y, ns.y);
-                }
+              for (int e = 0; e < 8; e += 2) {
+                // (cos, sin) of two pairs advanced by their steps, packed
+                const float4 st = *reinterpret_cast<const float4*>(rstep + 8 * c + e);
+                const float2 co = make_float2(cs[i][e].x, cs[i][e + 1].x);
+                const float2 si = make_float2(cs[i][e].y, cs[i][e + 1].y);
+                const float2 sc = make_float2(st.x, st.z), ss2 = make_float2(st.y, st.w);
+                const float2 nc = __ffma2_rn(co, sc, __fmul2_rn(si, make_float2(-ss2.x, -ss2.y)));
+                const float2 ns = __ffma2_rn(si, sc, __fmul2_rn(co, ss2));
+                cs[i][e] = make_float2(nc.x, ns.x);
+                cs[i][e + 1] = make_float2(nc.y, ns.y);
               }
             }
           }
