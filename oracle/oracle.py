@@ -123,15 +123,25 @@ def visible(i, j, window: int):
     return ok
 
 
-def _attend(qt, kt, vals, q_idx, k_idx, scale, cap, window):
-    """Softmax attention of transformed queries qt [R,D] over keys kt [N,D]."""
+def _attend(qt, kt, vals, q_idx, k_idx, scale, cap, window, valid=None):
+    """Softmax attention of transformed queries qt [R,D] over keys kt [N,D].
+
+    ``valid`` = (lo, hi) restricts the sequence to token indices [lo, hi): keys
+    outside it are masked, and a query outside it (a padding row) sees no key
+    and gets a zero output, as does any row with no visible key.
+    """
     s = (qt @ kt.T) * scale
     s = softcap(s, cap)
     mask = visible(q_idx[:, None], k_idx[None, :], window)
+    if valid is not None:
+        lo, hi = valid
+        mask = mask & (k_idx[None, :] >= lo) & (q_idx[:, None] >= lo) & (q_idx[:, None] < hi)
+    any_vis = mask.any(axis=1)
     s = np.where(mask, s, -np.inf)
-    m = np.max(s, axis=1, keepdims=True)
-    p = np.exp(s - m)
-    p = p / np.sum(p, axis=1, keepdims=True)
+    m = np.max(np.where(any_vis[:, None], s, 0.0), axis=1, keepdims=True)
+    p = np.where(mask, np.exp(s - m), 0.0)
+    den = np.sum(p, axis=1, keepdims=True)
+    p = p / np.where(den > 0, den, 1.0)
     return p @ vals
 
 
@@ -149,12 +159,17 @@ def _layer_fields(cfg):
 
 # --- the layer: prefill ------------------------------------------------------
 
-def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None):
+def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None, seq_range=None):
     """Self-attention forward over a whole prompt (float64).
 
     q [B,S,H,D], k [B,S,Hkv,D], v [B,S,Hkv,D] or None when cfg.k_eq_v,
     positions [B,S] (drive RoPE only).  ``rows`` optionally restricts the
-    output to those query indices (same for every b, h).  Returns [B,R,H,D].
+    output to those query indices (same for every b, h).  ``seq_range``
+    [B,2] optionally gives each sequence's valid tokens [lo, hi) (a padded
+    batch: KerasFormers "Gemma 4", Gemma4Generate.generate argument table,
+    `attention_mask` 1 = keep, 0 = padding, and its batched-prompt example); a
+    padding token is neither a query nor a key, and padding rows are zero.
+    Returns [B,R,H,D].
     """
     f = _layer_fields(cfg)
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -175,8 +190,9 @@ def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None):
                   f["rot"], f["theta"], f["F"])                      # [R,H,D]
         for h in range(H):
             kv = h // G
+            valid = None if seq_range is None else (int(seq_range[b][0]), int(seq_range[b][1]))
             out[b, :, h] = _attend(qt[:, h], kt[:, kv], vals_all[b, :, kv], rows, k_idx,
-                                   f["scale"], f["cap"], f["W"])
+                                   f["scale"], f["cap"], f["W"], valid)
     return out
 
 

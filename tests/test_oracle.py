@@ -368,3 +368,62 @@ def test_workloads_use_model_card_constants():
         g["gemma4_partial_rotary_factor"], g["gemma4_k_eq_v"])
     assert (d4l.num_kv_heads, d4l.head_dim, d4l.window) == (
         g["gemma4_num_kv_heads"], g["gemma4_head_dim"], g["gemma4_sliding_window"])
+
+
+# --- padded batches: each sequence's valid tokens [lo, hi) (KerasFormers "Gemma 4",
+# Gemma4Generate.generate: attention_mask 1 = keep, 0 = padding) ---------------------
+
+def test_seq_range_full_equals_unpadded():
+    B, S, D = 2, 9, 8
+    q, k, v = rnd((B, S, 2, D), 40), rnd((B, S, 1, D), 41), rnd((B, S, 1, D), 42)
+    pos = np.tile(np.arange(S), (B, 1))
+    for W in (0, 3):
+        cfg = layer(num_heads=2, head_dim=D, window=W, rotary_fraction=1.0)
+        full = O.attention_prefill(q, k, v, pos, cfg)
+        rng = np.array([[0, S]] * B)
+        assert np.array_equal(O.attention_prefill(q, k, v, pos, cfg, seq_range=rng), full)
+
+
+@pytest.mark.parametrize("W", [0, 1, 4])
+def test_left_padding_equals_sequence_alone(W):
+    # a sequence of n tokens placed after S - n padding tokens (garbage values,
+    # any positions), with range [S - n, S), gives on its rows what it gives alone
+    S, n, D = 11, 7, 8
+    x_q, x_k, x_v = rnd((1, n, 2, D), 43), rnd((1, n, 1, D), 44), rnd((1, n, 1, D), 45)
+    cfg = layer(num_heads=2, head_dim=D, window=W, rotary_fraction=0.5, rope_theta=100.0)
+    alone = O.attention_prefill(x_q, x_k, x_v, np.arange(n)[None], cfg)[0]
+    pad = S - n
+    q = np.concatenate([rnd((1, pad, 2, D), 46) * 100, x_q], axis=1)
+    k = np.concatenate([rnd((1, pad, 1, D), 47) * 100, x_k], axis=1)
+    v = np.concatenate([rnd((1, pad, 1, D), 48) * 100, x_v], axis=1)
+    pos = np.concatenate([np.full(pad, 3), np.arange(n)])[None]
+    got = O.attention_prefill(q, k, v, pos, cfg, seq_range=np.array([[pad, S]]))[0]
+    assert np.max(np.abs(got[pad:] - alone)) < 1e-12
+    assert np.all(got[:pad] == 0.0)
+
+
+def test_right_padding_rows_zero_and_rest_causal():
+    S, n, D = 10, 6, 4
+    q, k, v = rnd((1, S, 1, D), 49), rnd((1, S, 1, D), 50), rnd((1, S, 1, D), 51)
+    pos = np.arange(S)[None]
+    cfg = layer(head_dim=D)
+    full = O.attention_prefill(q, k, v, pos, cfg)[0]
+    got = O.attention_prefill(q, k, v, pos, cfg, seq_range=np.array([[0, n]]))[0]
+    assert np.array_equal(got[:n], full[:n])  # causal rows never see keys >= n
+    assert np.all(got[n:] == 0.0)
+
+
+def test_padding_onehot_probe_counts():
+    # q = 0: uniform weights over exactly the keys j with max(lo, i-W+1) <= j <= i
+    S, D = 9, 9
+    qz, kk, v = np.zeros((1, S, 1, D)), rnd((1, S, 1, D), 52), np.eye(S, D)[None, :, None, :]
+    for lo in range(0, S):
+        for W in (0, 2, 5):
+            wts = O.attention_prefill(qz, kk, v, np.arange(S)[None], layer(head_dim=D, window=W),
+                                      seq_range=np.array([[lo, S]]))[0, :, 0]
+            for i in range(S):
+                expect = np.zeros(S)
+                if i >= lo:
+                    first = lo if W == 0 else max(lo, i - W + 1)
+                    expect[first:i + 1] = 1.0 / (i + 1 - first)
+                assert np.max(np.abs(wts[i] - expect)) < 1e-15, (lo, W, i)

@@ -55,8 +55,15 @@ MUTATIONS = {
         "np.array([L - 1]),\n                  f[\"rot\"]", "np.array([L]),\n                  f[\"rot\"]",
         [T.test_decode_equals_last_prefill_row]),
     "softmax_drops_normaliser": (
-        "p = p / np.sum(p, axis=1, keepdims=True)", "p = p",
+        "p = p / np.where(den > 0, den, 1.0)", "p = p",
         [T.test_softmax_of_constant_values, T.test_worked_three_tokens]),
+    "padding_keys_not_masked": (
+        "mask = mask & (k_idx[None, :] >= lo) & (q_idx[:, None] >= lo)",
+        "mask = mask & (q_idx[:, None] >= lo)",
+        [T.test_left_padding_equals_sequence_alone, T.test_padding_onehot_probe_counts]),
+    "padding_rows_not_zeroed": (
+        "& (q_idx[:, None] >= lo) & (q_idx[:, None] < hi)", "",
+        [T.test_right_padding_rows_zero_and_rest_causal]),
 }
 
 
