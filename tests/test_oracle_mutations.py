@@ -45,7 +45,7 @@ MUTATIONS = {
         "return c * np.tanh(s / c)", "return np.tanh(s / c)",
         [T.test_softcap_closed_form]),
     "gqa_heads_strided": (
-        "            kv = h // G\n            out[b, :, h]", "            kv = h % Hkv\n            out[b, :, h]",
+        "            kv = h // G\n            valid", "            kv = h % Hkv\n            valid",
         [T.test_mqa_equals_replicated_gqa]),
     "keqv_values_are_normed_keys": (
         "vals_all = k if f[\"k_eq_v\"] else v",
