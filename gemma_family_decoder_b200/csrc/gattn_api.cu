@@ -234,10 +234,35 @@ size_t gattn_prefill_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t
   return bytes;
 }
 
+static int prefill_impl(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
+                        const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,
+                        int32_t batch, int32_t seq_len, const gattn_cfg* cfg, void* workspace,
+                        size_t ws_bytes, gattn_stream stream);
+
 int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
                   const int32_t* positions, gattn_bf16* out, int32_t batch, int32_t seq_len,
                   const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream) {
   g_last_error[0] = 0;
+  return prefill_impl(q, k, v_or_null, positions, nullptr, out, batch, seq_len, cfg, workspace, ws_bytes,
+                      stream);
+}
+
+int gattn_prefill_padded(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
+                         const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,
+                         int32_t batch, int32_t seq_len, const gattn_cfg* cfg, void* workspace,
+                         size_t ws_bytes, gattn_stream stream) {
+  g_last_error[0] = 0;
+  if (!seq_range) return fail(GATTN_ERR_INVALID_ARG, "seq_range must not be NULL");
+  if (reinterpret_cast<uintptr_t>(seq_range) & 3u)
+    return fail(GATTN_ERR_INVALID_ARG, "seq_range must be 4-byte aligned");
+  return prefill_impl(q, k, v_or_null, positions, seq_range, out, batch, seq_len, cfg, workspace, ws_bytes,
+                      stream);
+}
+
+static int prefill_impl(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
+                        const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,
+                        int32_t batch, int32_t seq_len, const gattn_cfg* cfg, void* workspace,
+                        size_t ws_bytes, gattn_stream stream) {
   gattn::LayerArgs la;
   int st = resolve(cfg, &la, true);
   if (st != GATTN_OK) return st;
@@ -289,6 +314,7 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
   pa.timeout_ns = gattn::wait_timeout_ns();
   pa.trace = static_cast<unsigned long long*>(g_trace_buf);
   pa.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
+  pa.seq_range = seq_range;
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
   cudaError_t e = gattn::launch_prefill(pa, la, s);
   if (g_prof_stop) cudaEventRecord(g_prof_stop, s);

@@ -84,6 +84,7 @@ struct PrefillArgs {
   uint64_t timeout_ns;
   unsigned long long* trace;  // optional kernel timeline buffer (null = off)
   size_t trace_bytes;
+  const int* seq_range = nullptr;  // [B][2] valid tokens of each sequence (padded batch), or null
 };
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
 

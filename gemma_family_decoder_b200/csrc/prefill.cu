@@ -74,6 +74,7 @@ struct PrefillKParams {
   LayerArgs la;
   unsigned long long* trace;  // optional per-CTA event times (kTraceSlots each), or null
   int trace_ctas;
+  const int* seq_range;       // [B][2] valid tokens [lo, hi) of each sequence, or null (all valid)
 };
 
 // Optional timeline of one CTA's first item (debug aid, off unless a trace
@@ -86,7 +87,9 @@ constexpr int kTraceSlots = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D, int BN, bool CAP>
+// PAD: the batch is padded (P.seq_range set); a separate instance so that the
+// unpadded kernel carries none of the extra masking
+template <int D, int BN, bool CAP, bool PAD>
 __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ PrefillKParams P) {
   using C = PrefillShape<D, BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -114,6 +117,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   // work item `it`, heaviest query tiles first
   struct Item {
     int qt, dvs, h, b, kvh, q0, dv_lo, k_first, ntiles, rot;
+    int lo, hi;  // the sequence's valid tokens (all of [0, S) unless the batch is padded)
   };
   auto item_of = [&](int it) {
     Item w;
@@ -127,10 +131,20 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     w.kvh = w.h / la.G;
     w.q0 = w.qt * C::BM;
     w.dv_lo = w.dvs * C::DV;
-    const int kv_hi = min(S, w.q0 + C::BM);
-    const int kv_lo = la.window > 0 ? max(0, w.q0 - la.window + 1) : 0;
+    w.lo = 0;
+    w.hi = S;
+    if constexpr (PAD) {
+      w.lo = min(max(__ldg(P.seq_range + 2 * w.b), 0), S);
+      w.hi = min(max(__ldg(P.seq_range + 2 * w.b + 1), 0), S);
+    }
+    // keys of the tile's valid rows: from the window's (and the sequence's)
+    // first key to the last valid row
+    const int kv_hi = min(min(S, w.q0 + C::BM), w.hi);
+    const int kv_lo = max(la.window > 0 ? max(0, w.q0 - la.window + 1) : 0, w.lo);
     w.k_first = (kv_lo / BN) * BN;
-    w.ntiles = (kv_hi - w.k_first + BN - 1) / BN;
+    // a query tile with no valid row reads no keys: its rows are zero
+    const bool none = PAD && (w.lo >= w.hi || w.q0 + C::BM <= w.lo || w.q0 >= w.hi);
+    w.ntiles = none ? 0 : (kv_hi - w.k_first + BN - 1) / BN;
     // KV tiles are visited starting at a tile that differs between the items
     // working on one sequence at once, so they do not all read the same L2
     // lines together (the online softmax is independent of the visiting order)
@@ -211,7 +225,20 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       if (it >= nitems) continue;
       const Item w = item_of(it);
       const int qi = w.q0 + t;
-      const bool valid = qi < S;
+      const bool in_seq = qi < S;                            // a row of the output
+      const bool valid = in_seq && (!PAD || (qi >= w.lo && qi < w.hi));  // and not padding
+      if (PAD && t == 0 && w.qt == 0 && w.h == 0 && w.dvs == 0) {
+        const int lo_in = __ldg(P.seq_range + 2 * w.b), hi_in = __ldg(P.seq_range + 2 * w.b + 1);
+        if (lo_in < 0 || hi_in > S) flag_status(P.status, kStatusBounds);
+      }
+      if (PAD && w.ntiles == 0) {
+        // every row of the tile is padding: zero output, no keys, no MMAs
+        if (in_seq) {
+          uint4* orow = reinterpret_cast<uint4*>(P.out + ((static_cast<size_t>(w.b) * S + qi) * H + w.h) * D + w.dv_lo);
+          for (int c = 0; c < C::DV / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < w.ntiles && ok; ++j) {
         const int T = T0 + j;
@@ -226,7 +253,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         tmem_wait_ld();
 
         const int key0 = tile_key(w, j);
-        const bool full_tile = (key0 + BN - 1 <= w.q0) && (w.q0 + C::BM <= S) &&
+        const bool full_tile = (key0 + BN - 1 <= w.q0) && (w.q0 + C::BM <= (PAD ? min(S, w.hi) : S)) &&
+                               (!PAD || (key0 >= w.lo && w.q0 >= w.lo)) &&
                                (W <= 0 || (w.q0 + C::BM - 1) - key0 < W);
         float x[BN];
 #pragma unroll
@@ -236,7 +264,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         }
         if (!full_tile) {
           const int hi = valid ? qi - key0 : -1;            // visible iff i <= hi
-          const int lo = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
+          const int lo_w = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
+          const int lo = PAD ? max(lo_w, w.lo - key0) : lo_w;
 #pragma unroll
           for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
         }
@@ -318,13 +347,13 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         uint4* orow = reinterpret_cast<uint4*>(
-            P.out + ((static_cast<size_t>(w.b) * S + (valid ? qi : 0)) * H + w.h) * D + w.dv_lo);
+            P.out + ((static_cast<size_t>(w.b) * S + (in_seq ? qi : 0)) * H + w.h) * D + w.dv_lo);
 #pragma unroll 1
         for (int c = 0; c < C::DV / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
           tmem_wait_ld();
-          if (valid) {
+          if (in_seq) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 u;
@@ -372,6 +401,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       const int it = item_at(r);
       if (it >= nitems) continue;
         const Item w = item_of(it);
+        if (PAD && w.ntiles == 0) continue;  // all padding: nothing to load
         ok = load_k(w, T0, 0);
         if (!ok) break;
         lk = T0;
@@ -453,6 +483,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       const int it = item_at(r);
       if (it >= nitems) continue;
         const Item w = item_of(it);
+        if (PAD && w.ntiles == 0) continue;  // all padding: nothing to multiply
         ok = mbar_wait(q_full, I & 1, tmo, P.status, abort_flag);
         if (!ok) break;
         if (I == 0) mark(3);
@@ -482,7 +513,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   if (threadIdx.x == 0) mark(5);
 }
 
-template <int D, int BN, bool CAP>
+template <int D, int BN, bool CAP, bool PAD>
 static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   using C = PrefillShape<D, BN>;
   PrefillKParams P;
@@ -500,7 +531,8 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.la = la;
   P.trace = pa.trace;
   P.trace_ctas = static_cast<int>(pa.trace_bytes / (kTraceSlots * sizeof(unsigned long long)));
-  auto kern = prefill_kernel<D, BN, CAP>;
+  P.seq_range = pa.seq_range;
+  auto kern = prefill_kernel<D, BN, CAP, PAD>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -520,10 +552,17 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
 
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   const bool cap = la.softcap > 0.f;
+  if (pa.seq_range) {
+    if (la.D == 256)
+      return cap ? run_prefill<256, 128, true, true>(pa, la, s) : run_prefill<256, 128, false, true>(pa, la, s);
+    if (la.D == 512)
+      return cap ? run_prefill<512, 64, true, true>(pa, la, s) : run_prefill<512, 64, false, true>(pa, la, s);
+    return cudaErrorInvalidValue;
+  }
   if (la.D == 256)
-    return cap ? run_prefill<256, 128, true>(pa, la, s) : run_prefill<256, 128, false>(pa, la, s);
+    return cap ? run_prefill<256, 128, true, false>(pa, la, s) : run_prefill<256, 128, false, false>(pa, la, s);
   if (la.D == 512)
-    return cap ? run_prefill<512, 64, true>(pa, la, s) : run_prefill<512, 64, false>(pa, la, s);
+    return cap ? run_prefill<512, 64, true, false>(pa, la, s) : run_prefill<512, 64, false, false>(pa, la, s);
   return cudaErrorInvalidValue;
 }
 

@@ -27,7 +27,7 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_rope_table_fill", "gattn_workspace_init", "gattn_prefill_workspace_size",
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
-           "gattn_set_trace_buffer", "gattn_decode_noalloc")
+           "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded")
 
 
 class GattnError(RuntimeError):
@@ -100,6 +100,9 @@ def lib() -> ctypes.CDLL:
         L.gattn_set_trace_buffer.argtypes = [vp, sz]
         L.gattn_decode_noalloc.restype = ctypes.c_int
         L.gattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp]
+        L.gattn_prefill_padded.restype = ctypes.c_int
+        L.gattn_prefill_padded.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz,
+                                           vp]
         _lib = L
     return _lib
 
@@ -201,8 +204,11 @@ class AttentionLayer:
         return ws
 
     # -- the two entry points ---------------------------------------------------
-    def prefill(self, q, k, v=None, positions=None, out=None, workspace=None, stream=None):
-        """gattn_prefill: q [B,S,H,D], k/v [B,S,Hkv,D] bf16, positions [B,S] int32."""
+    def prefill(self, q, k, v=None, positions=None, out=None, workspace=None, stream=None, seq_range=None):
+        """gattn_prefill: q [B,S,H,D], k/v [B,S,Hkv,D] bf16, positions [B,S] int32.
+
+        With ``seq_range`` (int32 [B,2], sequence b's valid tokens [lo, hi)) this calls
+        gattn_prefill_padded: padding tokens are neither queries nor keys, their rows are zero."""
         _need(q, "q", torch.bfloat16, 4)
         _need(k, "k", torch.bfloat16, 4)
         if v is not None:
@@ -214,6 +220,15 @@ class AttentionLayer:
             _need(positions, "positions", torch.int32, 2)
         out = torch.empty_like(q) if out is None else out
         ws = self.prefill_workspace(B, S, q.device) if workspace is None else workspace
+        if seq_range is not None:
+            _need(seq_range, "seq_range", torch.int32, 2)
+            if tuple(seq_range.shape) != (B, 2):
+                raise ValueError(f"seq_range must be [{B}, 2], got {tuple(seq_range.shape)}")
+            _raise_if(lib().gattn_prefill_padded(_ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(seq_range),
+                                                 _ptr(out), B, S, ctypes.byref(self.cfg), _ptr(ws), ws.numel(),
+                                                 _stream(stream)),
+                      "gattn_prefill_padded")
+            return out
         _raise_if(lib().gattn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(positions), _ptr(out), B, S,
                                       ctypes.byref(self.cfg), _ptr(ws), ws.numel(), _stream(stream)),
                   "gattn_prefill")

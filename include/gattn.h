@@ -125,6 +125,26 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
                   const int32_t* positions, gattn_bf16* out, int32_t batch, int32_t seq_len,
                   const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream);
 
+/* ---- prefill of a padded batch ------------------------------------------------
+ * The same layer over a batch whose sequences are padded to seq_len: the
+ * batched-prompt `attention_mask` (1 = keep, 0 = padding) of KerasFormers
+ * "Gemma 4", Gemma4Generate.generate, given as each sequence's contiguous run
+ * of valid tokens.
+ *   seq_range [batch][2] int32 (device): valid tokens [lo, hi) of sequence b,
+ *             0 <= lo <= hi <= seq_len (left padding: lo > 0; right: hi < seq_len).
+ *             Values outside [0, seq_len] are clamped and flag
+ *             GATTN_ERR_DEVICE_BOUNDS; lo >= hi makes the whole sequence padding.
+ * A padding token is neither a query nor a key: key j is visible to query i
+ * iff lo <= j <= i < hi (and i - j < window when windowed), and the output
+ * rows of padding tokens are zero.  Positions of padding tokens must still be
+ * in [0, rope_max_pos) (they are rotated, then ignored).  Every other argument,
+ * the workspace size and the errors are those of gattn_prefill; with every
+ * range [0, seq_len) the result is bit-identical to gattn_prefill's. */
+int gattn_prefill_padded(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
+                         const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,
+                         int32_t batch, int32_t seq_len, const gattn_cfg* cfg, void* workspace,
+                         size_t ws_bytes, gattn_stream stream);
+
 /* ---- decode ----------------------------------------------------------------
  * One decode step: query b (at position seq_lens[b]-1) against cache rows
  * [0, seq_lens[b]) of its own cache.  Caches hold RAW keys/values (before

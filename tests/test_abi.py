@@ -90,6 +90,24 @@ def test_prefill_rejects_bad_pointers_and_sizes():
     assert prefill(cr, pos=None) == INVALID
 
 
+def prefill_padded(c, sr=ALIGNED, B=1, S=16, **kw):
+    a = dict(q=ALIGNED, k=ALIGNED, v=ALIGNED, pos=ALIGNED, out=ALIGNED, ws=ALIGNED, ws_bytes=1 << 30)
+    a.update(kw)
+    return G.lib().gattn_prefill_padded(a["q"], a["k"], a["v"], a["pos"], sr, a["out"], B, S, ctypes.byref(c),
+                                        a["ws"], a["ws_bytes"], None)
+
+
+def test_prefill_padded_rejects_bad_args():
+    c = cfg()
+    assert prefill_padded(c, sr=None) == INVALID
+    assert prefill_padded(c, sr=ALIGNED + 2) == INVALID      # int32 pairs: 4-byte aligned
+    assert prefill_padded(c, q=ALIGNED + 8) == INVALID       # then every check of gattn_prefill
+    assert prefill_padded(c, ws_bytes=16) == WORKSPACE
+    assert prefill_padded(cfg(head_dim=128)) == UNSUPPORTED
+    assert prefill_padded(c, B=0) == 0
+    assert G.lib().gattn_last_error() == b""
+
+
 def test_empty_problem_is_a_no_op():
     assert prefill(cfg(), B=0) == 0
     assert prefill(cfg(), S=0) == 0
