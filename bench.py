@@ -43,6 +43,7 @@ PREFILL_WL = {
     "gemma3_1b_local_w512_b2_s8192": W.GEMMA3_LOCAL,
     "gemma3_1b_global_b2_s8192": W.GEMMA3_GLOBAL,
     "gemma4_12b_global_keqv_s32768": W.GEMMA4_GLOBAL,
+    "gemma3_1b_global_b8_s4096_leftpad": W.GEMMA3_GLOBAL_LEFTPAD,
 }
 DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
                                  W.GEMMA4_DECODE_GLOBAL_NORM)}
@@ -64,9 +65,28 @@ def row_visible(i, window):
     return i + 1 if window <= 0 else np.minimum(i + 1, window)
 
 
-def prefill_flops(wl: W.PrefillWorkload) -> float:
+def prefill_flops(wl: W.PrefillWorkload, seq_range=None) -> float:
+    """Q K^T and P V multiply-adds (2 FLOPs each) over the visible pairs; a padded batch
+    counts each sequence's valid tokens only."""
     L = wl.layer
-    return 4.0 * L.head_dim * L.num_heads * wl.batch * visible_pairs(wl.seq, L.window)
+    if seq_range is None:
+        return 4.0 * L.head_dim * L.num_heads * wl.batch * visible_pairs(wl.seq, L.window)
+    pairs = sum(visible_pairs(int(hi) - int(lo), L.window) for lo, hi in seq_range.tolist() if hi > lo)
+    return 4.0 * L.head_dim * L.num_heads * pairs
+
+
+def rows_flops(wl: W.PrefillWorkload, d, rows) -> float:
+    """FLOPs of the query rows ``rows`` of every sequence (padding rows count nothing)."""
+    L = wl.layer
+    rows = np.asarray(rows, dtype=np.int64)
+    sr = d.get("seq_range")
+    if sr is None:
+        return 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(rows, L.window).sum())
+    total = 0.0
+    for lo, hi in sr.tolist():
+        r = rows[(rows >= lo) & (rows < hi)]
+        total += float(row_visible(r - lo, L.window).sum())
+    return 4.0 * L.head_dim * L.num_heads * total
 
 
 def decode_bytes(layer: W.Layer, seq_lens) -> float:
@@ -208,17 +228,18 @@ def make_prefill(wl, dev):
     from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
     d = W.prefill_inputs(wl)
     layer = AttentionLayer(LayerSpec.of(wl.layer), wl.seq, d["w_q"], d["w_k"], device=dev)
-    host = {k: d[k].pin_memory() for k in ("q", "k", "v", "positions") if d[k] is not None}
+    host = {k: d[k].pin_memory() for k in ("q", "k", "v", "positions", "seq_range") if d[k] is not None}
     devt = {k: t.to(dev) for k, t in host.items()}
     out = torch.empty_like(devt["q"])
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     ws = layer.prefill_workspace(wl.batch, wl.seq, dev)
 
     def step(src=devt):
-        layer.prefill(src["q"], src["k"], src.get("v"), src["positions"], out=out, workspace=ws)
+        layer.prefill(src["q"], src["k"], src.get("v"), src["positions"], out=out, workspace=ws,
+                      seq_range=src.get("seq_range"))
 
     return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
-                work=prefill_flops(wl), unit="TFLOP/s", scale=1e12,
+                work=prefill_flops(wl, d["seq_range"]), unit="TFLOP/s", scale=1e12,
                 metric="attention prefill TFLOP/s (effective FLOPs)", bound="tensor",
                 launches=2 if (wl.layer.rot_dim or wl.layer.qk_norm) else 1,
                 kernel_src=("gemma_family_decoder_b200/csrc/prefill.cu",
@@ -401,7 +422,7 @@ def run_ours(args, world, rank, local):
 def _oracle_prefill_rows(wl, d, rows):
     import oracle as O
     O.attention_prefill(d["q"], d["k"], d["v"], d["positions"], wl.layer, w_q=d["w_q"],
-                        w_k=d["w_k"], rows=rows)
+                        w_k=d["w_k"], rows=rows, seq_range=d.get("seq_range"))
 
 
 def cpu_baseline(name, budget_s=15.0):
@@ -422,7 +443,7 @@ def cpu_baseline(name, budget_s=15.0):
         _oracle_prefill_rows(wl, d, rows)
         dt = time.perf_counter() - t0
         L = wl.layer
-        work = 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(rows, L.window).sum())
+        work = rows_flops(wl, d, rows)
         return {"value": round(work / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
                 "kind": "oracle",
                 "sample": f"{len(rows)} evenly spaced query rows of {S}, all {wl.batch} sequences and "
@@ -477,7 +498,7 @@ def run_reference(args, world, rank):
             el = time.perf_counter() - t0
             if i >= args.warmup:
                 dt += el
-                work += 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(rows, L.window).sum())
+                work += rows_flops(wl, d, rows)
         value, unit = work / dt / 1e12, "TFLOP/s"
         sample = f"{rows_per_step} random query rows of {S} per step, all sequences and heads"
         metric = "attention prefill TFLOP/s (effective FLOPs)"

@@ -167,3 +167,29 @@ def test_out_of_range_seq_range_is_flagged_and_clamped():
     ref = O.attention_prefill(d["q"], d["k"], d["v"], d["positions"], layer, seq_range=clamped)
     assert_close(out, ref, "clamped")
     check_padding_rows_zero(out, clamped)
+
+
+def test_leftpad_workload_sampled_rows():
+    # the benchmarked left-padded batch at full size: rows on both sides of every
+    # sequence's first kept token, the first and last tiles, and random rows
+    wl = W.GEMMA3_GLOBAL_LEFTPAD
+    d = W.prefill_inputs(wl)
+    ranges = d["seq_range"].tolist()
+    S = wl.seq
+    L = make_layer(wl.layer, S, d["w_q"], d["w_k"])
+    dv = to_dev(d, keys=("q", "k", "v", "positions", "seq_range"))
+    ws = L.prefill_workspace(wl.batch, S)
+    out = L.prefill(dv["q"], dv["k"], dv["v"], dv["positions"], workspace=ws, seq_range=dv["seq_range"])
+    from gemma_family_decoder_b200 import check
+    assert check(ws) == 0
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(wl.seed)
+    rows = {0, 127, 128, S - 129, S - 1} | set(int(r) for r in rng.integers(0, S, 6))
+    for lo, _ in ranges:
+        rows |= {max(0, lo - 1), lo, min(S - 1, lo + 1), min(S - 1, lo + 200)}
+    rows = np.array(sorted(rows))
+    ref = O.attention_prefill(d["q"], d["k"], d["v"], d["positions"], wl.layer, w_q=d["w_q"], w_k=d["w_k"],
+                              rows=rows, seq_range=ranges)
+    got = out[:, torch.as_tensor(rows, device=out.device)]
+    assert_close(got, ref, wl.name)
+    check_padding_rows_zero(out, ranges)

@@ -70,6 +70,9 @@ class PrefillWorkload:
     seed: int
     gain_mean: float = 0.0   # w ~ gain_mean + N(0, gain_std)
     gain_std: float = 0.1
+    # > 0: a left-padded batch of prompts (KerasFormers "Gemma 4", Gemma4Generate.generate,
+    # attention_mask), sequence b holding the last n_b tokens, n_b ~ U[len_lo, seq]
+    len_lo: int = 0
 
 
 @dataclasses.dataclass(frozen=True)
@@ -136,8 +139,14 @@ GEMMA4_DECODE_GLOBAL_NORM = DecodeWorkload(
     dataclasses.replace(GEMMA4_DECODE_GLOBAL.layer, qk_norm=NORM_W),
     batch=64, len_lo=1024, len_hi=32768, seed=4, gain_mean=1.0, gain_std=0.1)
 
+# a batch of eight prompts of 512 to 4096 tokens, left-padded to 4096, through the
+# Gemma 3 global layer
+GEMMA3_GLOBAL_LEFTPAD = PrefillWorkload(
+    "gemma3_1b_global_b8_s4096_leftpad",
+    Layer(window=0, rope_theta=1e6, **_G3), batch=8, seq=4096, seed=5, len_lo=512)
+
 PREFILL: Dict[str, PrefillWorkload] = {w.name: w for w in (
-    GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL)}
+    GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL, GEMMA3_GLOBAL_LEFTPAD)}
 DECODE: Dict[str, DecodeWorkload] = {w.name: w for w in (
     GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM)}
 
@@ -174,7 +183,18 @@ def prefill_inputs(wl: PrefillWorkload, batch: Optional[int] = None,
     v = None if layer.k_eq_v else _randn_bf16(gen, (B, S, Hkv, D))
     w_q, w_k = _gains(gen, layer, wl.gain_mean, wl.gain_std)
     positions = torch.arange(S, dtype=torch.int32).unsqueeze(0).repeat(B, 1)
-    return dict(q=q, k=k, v=v, positions=positions, w_q=w_q, w_k=w_k, layer=layer)
+    seq_range = None
+    if wl.len_lo > 0:
+        # left padding: sequence b keeps tokens [S - n_b, S), numbered 0, 1, ... from the
+        # first kept one; padding tokens sit at position 0 (a shorter S scales len_lo)
+        n_lo = max(1, wl.len_lo * S // wl.seq)
+        n = torch.randint(n_lo, S + 1, (B,), generator=gen, dtype=torch.int64)
+        lo = (S - n).to(torch.int32)
+        seq_range = torch.stack([lo, torch.full_like(lo, S)], dim=1).contiguous()
+        t = torch.arange(S, dtype=torch.int32).unsqueeze(0)
+        positions = torch.clamp(t - lo.unsqueeze(1), min=0).to(torch.int32).contiguous()
+    return dict(q=q, k=k, v=v, positions=positions, w_q=w_q, w_k=w_k, layer=layer,
+                seq_range=seq_range)
 
 
 def decode_inputs(wl: DecodeWorkload, batch: Optional[int] = None,
