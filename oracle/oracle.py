@@ -25,6 +25,9 @@ widened) bf16 input values, in the order the layer applies them:
    key and value projections tied).
 7. GQA/MQA head grouping: query head h reads kv head h // (H / Hkv)
    (KerasFormers "Gemma" API num_kv_heads=1; ZeroModels "Gemma 2" GQA bullet).
+8. An int8 KV cache (Atlas "Gemma 4" summary, long-context/KV section: int8 KV
+   caching, Table 3 "+KV"): per-row symmetric codes and an fp32 scale,
+   dequantised before step 1 (``kv_quantize``, ``attention_decode_int8``).
 
 Readings taken where the pages are silent (each is listed in the design doc):
 scale = scalar**-0.5; softcap after scaling; norm before RoPE; V is the raw k
@@ -254,3 +257,46 @@ def chunk_partial(s, vals):
     m = np.max(s)
     p = np.exp(s - m)
     return m, np.sum(p), p @ vals
+
+
+# --- int8 KV cache ---------------------------------------------------------------
+
+def kv_quantize(x):
+    """Symmetric int8 codes of cache rows, one fp32 scale per row (float32 arithmetic).
+
+    The Atlas summary of the Gemma 4 report lists int8 KV caching (Table 3, "+KV")
+    without its format; the reading here: each row x (the head_dim values of one
+    position and kv head) gets scale s = max|x| / 127 and codes
+    c = round-half-even(x / s) clipped to [-127, 127], so that c * s is the
+    dequantised row.  Both divisions are IEEE float32 (correctly rounded): the
+    codes are integers decided by floating point, so the precision is fixed here.
+    A row of zeros gets s = 0 and codes 0.  x [..., D] -> (int8 [..., D], fp32 [...]).
+    """
+    x = np.asarray(_f64(x), dtype=np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    c = np.rint((x / safe[..., None]).astype(np.float32))
+    c = np.clip(c, -127, 127)
+    c = np.where((s > 0)[..., None], c, 0.0)
+    return c.astype(np.int8), s
+
+
+def kv_dequantize(codes, scales):
+    """codes [..., D] int8 times their row's scale [...], in float64."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def attention_decode_int8(q, k_codes, k_scales, v_codes, v_scales, seq_lens, cfg, w_q=None, w_k=None,
+                          batches=None, first_rows=None):
+    """One decode step over an int8 cache: attention_decode on the dequantised rows.
+
+    k_codes / v_codes [B,Lmax,Hkv,D] int8 (or per-batch lists, as attention_decode
+    takes), k_scales / v_scales [B,Lmax,Hkv] (or lists); with K=V the values are
+    the dequantised raw keys (v_codes / v_scales unused).
+    """
+    f = _layer_fields(cfg)
+    kd = [kv_dequantize(k_codes[b], k_scales[b]) for b in range(len(k_codes))]
+    vd = None if f["k_eq_v"] else [kv_dequantize(v_codes[b], v_scales[b]) for b in range(len(v_codes))]
+    return attention_decode(q, kd, vd, seq_lens, cfg, w_q=w_q, w_k=w_k, batches=batches,
+                            first_rows=first_rows)

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import oracle.oracle as src_mod
 import test_oracle as T
+import test_oracle_int8 as T8
 
 MUTATIONS = {
     # name: (original text, replacement, pins that must fail)
@@ -64,6 +65,25 @@ MUTATIONS = {
     "padding_rows_not_zeroed": (
         "& (q_idx[:, None] >= lo) & (q_idx[:, None] < hi)", "",
         [T.test_right_padding_rows_zero_and_rest_causal]),
+    "int8_scale_over_128": (
+        "amax / np.float32(127.0)", "amax / np.float32(128.0)",
+        [T8.test_exact_on_codes_times_power_of_two]),
+    "int8_codes_truncated": (
+        "c = np.rint((x / safe[..., None]).astype(np.float32))",
+        "c = np.trunc((x / safe[..., None]).astype(np.float32))",
+        [T8.test_codes_are_nearest_integers_brute_force, T8.test_exact_halves_round_to_even]),
+    "int8_ties_away_from_zero": (
+        "c = np.rint((x / safe[..., None]).astype(np.float32))",
+        "c = np.floor((x / safe[..., None]).astype(np.float32) + 0.5)",
+        [T8.test_exact_halves_round_to_even]),
+    "int8_dequant_drops_scale": (
+        "return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]",
+        "return np.asarray(codes, dtype=np.float64)",
+        [T8.test_round_trip_within_half_step_and_extremes,
+         T8.test_int8_decode_equals_float_decode_on_representable_cache]),
+    "int8_values_from_key_codes": (
+        "[kv_dequantize(v_codes[b], v_scales[b])", "[kv_dequantize(k_codes[b], v_scales[b])",
+        [T8.test_int8_decode_equals_float_decode_on_representable_cache]),
 }
 
 
