@@ -46,7 +46,7 @@ PREFILL_WL = {
     "gemma3_1b_global_b8_s4096_leftpad": W.GEMMA3_GLOBAL_LEFTPAD,
 }
 DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
-                                 W.GEMMA4_DECODE_GLOBAL_NORM)}
+                                 W.GEMMA4_DECODE_GLOBAL_NORM, W.GEMMA4_DECODE_LOCAL_INT8)}
 HEADLINE = "gemma1_2b_mqa_b4_s2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -89,11 +89,13 @@ def rows_flops(wl: W.PrefillWorkload, d, rows) -> float:
     return 4.0 * L.head_dim * L.num_heads * total
 
 
-def decode_bytes(layer: W.Layer, seq_lens) -> float:
+def decode_bytes(layer: W.Layer, seq_lens, int8: bool = False) -> float:
+    """Bytes a decode step must move: the visible cache rows (bf16, or int8 codes plus one
+    fp32 scale per row and kv head), the query and the output."""
     n = np.asarray(seq_lens, dtype=np.int64)
     if layer.window > 0:
         n = np.minimum(n, layer.window)
-    per_row = layer.num_kv_heads * layer.head_dim * 2
+    per_row = layer.num_kv_heads * (layer.head_dim + 4 if int8 else layer.head_dim * 2)
     kv = n.sum() * per_row * (1 if layer.k_eq_v else 2)
     qo = len(n) * layer.num_heads * layer.head_dim * 2 * 2
     return float(kv + qo)
@@ -269,11 +271,22 @@ def make_decode(wl, dev):
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     ws = layer.decode_workspace(wl.batch, wl.max_len, dev)
 
-    def step(src=devt):
-        layer.decode(src["q"], devt["k"], devt["v"], src["seq_lens"], out=out, workspace=ws)
+    if wl.kv_int8:
+        from gemma_family_decoder_b200 import kv_quantize
+        kq, ks = kv_quantize(k)
+        vq, vs = (None, None) if v is None else kv_quantize(v)
+        del k, v
+        devt.update(k=None, v=None, kq=kq, ks=ks, vq=vq, vs=vs)
+
+        def step(src=devt):
+            layer.decode_int8(src["q"], devt["kq"], devt["ks"], devt["vq"], devt["vs"], src["seq_lens"], out=out,
+                              workspace=ws)
+    else:
+        def step(src=devt):
+            layer.decode(src["q"], devt["k"], devt["v"], src["seq_lens"], out=out, workspace=ws)
 
     return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
-                work=decode_bytes(L, lens.numpy()), unit="GB/s", scale=1e9,
+                work=decode_bytes(L, lens.numpy(), wl.kv_int8), unit="GB/s", scale=1e9,
                 metric="decode KV GB/s (algorithmic bytes)", bound="hbm", launches=2,
                 kernel_src=("gemma_family_decoder_b200/csrc/prep_decode.cu",
                             "gemma_family_decoder_b200/csrc/decode_tc.cu",
@@ -425,6 +438,32 @@ def _oracle_prefill_rows(wl, d, rows):
                         w_k=d["w_k"], rows=rows, seq_range=d.get("seq_range"))
 
 
+def _oracle_cache(wl, ks, vs):
+    """The oracle's cache rows per batch row (None where left out): bf16 as drawn, or, for an
+    int8 workload, the oracle's own codes and scales of them."""
+    import oracle as O
+    if not wl.kv_int8:
+        return dict(k=ks, v=vs)
+
+    def q8(rows):
+        cs = [None if r is None else O.kv_quantize(r.float().numpy()) for r in rows]
+        return [None if c is None else c[0] for c in cs], [None if c is None else c[1] for c in cs]
+
+    kc, ksc = q8(ks)
+    vc, vsc = (None, None) if wl.layer.k_eq_v else q8(vs)
+    return dict(kc=kc, ks=ksc, vc=vc, vs=vsc)
+
+
+def _oracle_decode(wl, dq, cache, batches, firsts):
+    import oracle as O
+    L = wl.layer
+    if wl.kv_int8:
+        return O.attention_decode_int8(dq["q"], cache["kc"], cache["ks"], cache["vc"], cache["vs"], dq["seq_lens"],
+                                       L, w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts)
+    return O.attention_decode(dq["q"], cache["k"], None if L.k_eq_v else cache["v"], dq["seq_lens"], L,
+                              w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts)
+
+
 def cpu_baseline(name, budget_s=15.0):
     """The oracle timed on a strided sample of query rows (prefill) or batch rows (decode)."""
     import oracle as O
@@ -460,15 +499,15 @@ def cpu_baseline(name, budget_s=15.0):
         ks.append(rows["k"])
         vs.append(rows["v"])
         firsts.append(lo)
+    cache = _oracle_cache(wl, ks, vs)
     t0 = time.perf_counter()
     for b in range(wl.batch):
-        O.attention_decode(dq["q"], ks, None if L.k_eq_v else vs, dq["seq_lens"], L, w_q=dq["w_q"],
-                           w_k=dq["w_k"], batches=[b], first_rows=firsts)
+        _oracle_decode(wl, dq, cache, [b], firsts)
         done.append(b)
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    work = decode_bytes(L, lens[done])
+    work = decode_bytes(L, lens[done], wl.kv_int8)
     return {"value": round(work / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{len(done)} of {wl.batch} batch rows ({dt:.1f} s, float64 numpy)"}
 
@@ -516,13 +555,13 @@ def run_reference(args, world, rank):
             ks = [rows["k"] if j == b else None for j in range(wl.batch)]
             vs = [rows["v"] if j == b else None for j in range(wl.batch)]
             fr = [lo if j == b else 0 for j in range(wl.batch)]
+            cache = _oracle_cache(wl, ks, vs)
             t0 = time.perf_counter()
-            O.attention_decode(dq["q"], ks, None if L.k_eq_v else vs, dq["seq_lens"], L,
-                               w_q=dq["w_q"], w_k=dq["w_k"], batches=[b], first_rows=fr)
+            _oracle_decode(wl, dq, cache, [b], fr)
             el = time.perf_counter() - t0
             if i >= args.warmup:
                 dt += el
-                work += decode_bytes(L, lens[b:b + 1])
+                work += decode_bytes(L, lens[b:b + 1], wl.kv_int8)
         value, unit = work / dt / 1e9, "GB/s"
         sample = "one batch row per step, cycling over the batch"
         metric = "decode KV GB/s (algorithmic bytes)"

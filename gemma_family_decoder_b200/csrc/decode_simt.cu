@@ -21,6 +21,12 @@
 //   online softmax runs on those, and P V reads the probabilities back from a
 //   per-warp scratch.
 //
+// * An int8 cache (Q8) keeps the tile's rows and positions but half the bytes,
+//   with more stages in flight.  Each warp copies the fp32 scales of its own
+//   rows of a tile (4-byte asynchronous copies, one commit group per tile,
+//   NST tiles ahead); the key scale multiplies the reduced logit (and, squared,
+//   the QK-norm sum of squares), the value scale the probability that P V reads.
+//
 // Output: the same (m, l, O) partial per (b, head, split) as the other decode
 // kernels, split = chunk * SUB + sub, merged by decode_combine_kernel.  Every
 // split slot of every sequence is written once: a real partial by the segment
@@ -38,32 +44,37 @@ namespace gattn {
 namespace {
 
 constexpr int kSW = 8;                  // compute warps
-constexpr int kTileBytes = 32768;       // cache bytes per tile (keys; values as many)
+constexpr int kTileBytes = 32768;       // bf16 cache bytes per tile (keys; values as many); int8: half
 constexpr int kTabBytes = 8192;         // RoPE table rows of a tile, staged when they fit
 constexpr int kPlanSMs = 148;           // work-item target for the split plan (B200 SM count)
 constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n >> 1); }
 
-template <int D, int G, bool KEQV>
+template <int D, int G, bool KEQV, bool Q8>
 struct SimtShape {
   static constexpr int NC = D / 128;                 // 4-dim groups per lane
+  static constexpr int ES = Q8 ? 1 : 2;              // bytes per cached value
   static constexpr int ROWS = kTileBytes / (2 * D);  // cache rows per tile
+  static constexpr int KT = ROWS * D * ES;           // bytes of a tile's key rows (value rows as many)
   static constexpr int RPW = ROWS / kSW;             // rows per warp per tile
   static constexpr int NV = RPW * G;                 // logits per warp per tile
   static constexpr int LOGNV = ilog2(NV);
   static constexpr int LOGG = ilog2(G);
-  static constexpr int OFF_TAB = KEQV ? kTileBytes : 2 * kTileBytes;  // the tile's RoPE table rows
+  static constexpr int OFF_TAB = KEQV ? KT : 2 * KT;  // the tile's RoPE table rows
   static constexpr int STAGE = OFF_TAB + kTabBytes;
-  static constexpr int NST = KEQV ? 5 : 3;
+  static constexpr int NST = Q8 ? (KEQV ? 8 : 5) : (KEQV ? 5 : 3);
   static constexpr int OFF_BAR = NST * STAGE;
   static constexpr int OFF_MISC = OFF_BAR + 2 * NST * 8;
   static constexpr int OFF_SCR = OFF_MISC + 16;      // per warp: p [32], 1/rms [8]
   static constexpr int SCR_FLOATS = 40;
-  static constexpr int SMEM = OFF_SCR + kSW * SCR_FLOATS * 4 + 128;  // + slack to align the base
+  static constexpr int OFF_SSC = OFF_SCR + kSW * SCR_FLOATS * 4;  // Q8, per warp: [NST][K, V][RPW] scales
+  static constexpr int SSC_FLOATS = Q8 ? NST * 2 * RPW : 0;
+  static constexpr int SMEM = OFF_SSC + kSW * SSC_FLOATS * 4 + 128;  // + slack to align the base
   static_assert(NV >= 2 && NV <= 32 && (NV & (NV - 1)) == 0, "logits per warp tile");
   static_assert(G * NC * 4 <= 32, "accumulator registers per lane");
   static_assert(RPW <= 8, "norm scratch");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
 };
 
 struct SimtParams {
@@ -218,6 +229,14 @@ __device__ __forceinline__ void load_lane2(const uint8_t* row, int lane, float2 
   }
 }
 
+// the same from an int8 row (x[c][i] = codes of dims 4 lane + 128 c + 2i, +1)
+template <int NC>
+__device__ __forceinline__ void load_lane_q8(const uint8_t* row, int lane, float2 (&x)[NC][2]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    unpack_i8x4(*reinterpret_cast<const uint32_t*>(row + 4 * lane + 128 * c), x[c][0], x[c][1]);
+}
+
 template <int NC>
 __device__ __forceinline__ void zero_lane2(float2 (&x)[NC][2]) {
 #pragma unroll
@@ -277,9 +296,9 @@ __device__ __forceinline__ void unpack_lane(const uint8_t* row, int lane, float 
 
 }  // namespace
 
-template <int D, int G, bool KEQV>
+template <int D, int G, bool KEQV, bool Q8>
 __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_constant__ SimtParams P) {
-  using C = SimtShape<D, G, KEQV>;
+  using C = SimtShape<D, G, KEQV, Q8>;
   constexpr int NC = C::NC, RPW = C::RPW, NV = C::NV;
   const DecodeArgs& da = P.da;
   const LayerArgs& la = P.la;
@@ -316,9 +335,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
   // Stage st of tile u is refilled with tile u + NST by the last warp to finish
   // tile u (one arrival counter per stage); warp 0 issues the first NST tiles.
   // Every warp walks the same cursor, NST tiles ahead of the tile it computes.
+  const uint8_t* kbase = Q8 ? reinterpret_cast<const uint8_t*>(da.kq) : reinterpret_cast<const uint8_t*>(da.k);
+  const uint8_t* vbase = Q8 ? reinterpret_cast<const uint8_t*>(da.vq) : reinterpret_cast<const uint8_t*>(da.v);
   auto issue = [&](int st, int b, int p0, int npos) {
-    const uint32_t bytes = static_cast<uint32_t>(npos * row_elems * sizeof(__nv_bfloat16));
-    const size_t off = (static_cast<size_t>(b) * da.max_len + p0) * row_elems;
+    const uint32_t bytes = static_cast<uint32_t>(npos * row_elems * C::ES);
+    const size_t off = (static_cast<size_t>(b) * da.max_len + p0) * row_elems * C::ES;
     // table rows past the table's end are not copied; their positions are
     // flagged and clamped by the compute loop
     const int trows = tab_staged ? max(0, min(npos, la.rope_max_pos - p0)) : 0;
@@ -326,20 +347,45 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
     uint8_t* dst = smem + st * C::STAGE;
     fence_proxy_async_smem();  // this stage's earlier reads come before the copies' writes
     mbar_arrive_expect_tx(&full[st], (KEQV ? bytes : 2 * bytes) + tbytes);
-    bulk_load(dst, da.k + off, bytes, &full[st]);
-    if (!KEQV) bulk_load(dst + kTileBytes, da.v + off, bytes, &full[st]);
+    bulk_load(dst, kbase + off, bytes, &full[st]);
+    if (!KEQV) bulk_load(dst + C::KT, vbase + off, bytes, &full[st]);
     if (tbytes) bulk_load(dst + C::OFF_TAB, la.rope_tab + static_cast<size_t>(p0) * half, tbytes, &full[st]);
+  };
+  const int kvh = warp % Hkv, sub = warp / Hkv;
+  // int8 cache: this warp's rows' scales of a tile into its slot st (a row
+  // past the tile's positions gets 0), as one commit group per tile
+  float* ssc = reinterpret_cast<float*>(smem + C::OFF_SSC) + warp * C::SSC_FLOATS;
+  auto copy_scales = [&](int st, int b, int p0, int npos) {
+    if constexpr (Q8) {
+      const int r = lane % C::RPW, kind = lane / C::RPW;  // kind 0: key scale, 1: value scale
+      if (lane < 2 * C::RPW && !(KEQV && kind == 1)) {
+        float* dst = ssc + (st * 2 + kind) * C::RPW + r;
+        const int pr = sub + r * SUB;
+        if (pr < npos)
+          cp_async4(dst, (kind ? da.vs : da.ks) + (static_cast<size_t>(b) * da.max_len + p0 + pr) * Hkv + kvh);
+        else
+          *dst = 0.f;
+      }
+      cp_async_commit();
+    }
   };
   TileCursor ahead;
   ahead.init(P, i0, i1, TP);
   {
-    int tb, tp0, tn;
-    for (int u = 0; u < C::NST && ahead.next(P, &tb, &tp0, &tn); ++u)
+    int tb, tp0, tn, u = 0;
+    for (; u < C::NST && ahead.next(P, &tb, &tp0, &tn); ++u) {
       if (warp == 0 && lane == 0) issue(u, tb, tp0, tn);
+      copy_scales(u, tb, tp0, tn);
+    }
+    if constexpr (Q8)
+      for (; u < C::NST; ++u) cp_async_commit();  // NST groups ahead, some empty
   }
 
   // -------------------------------------------------------------- compute
-  const int kvh = warp % Hkv, sub = warp / Hkv;
+  auto load_row = [&](const uint8_t* row, float2 (&x)[NC][2]) {
+    if constexpr (Q8) load_lane_q8<NC>(row, lane, x);
+    else load_lane2<NC>(row, lane, x);
+  };
   const int idx = transpose_index<NV>(lane);
   const int ih = idx % G, ir = idx / G;  // this lane's (row, head) after the butterfly
   float* scr = reinterpret_cast<float*>(smem + C::OFF_SCR) + warp * C::SCR_FLOATS;
@@ -432,11 +478,17 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
         ok = false;
         break;
       }
+      if constexpr (Q8) {
+        cp_async_wait<C::NST - 1>();  // this tile's scales (group t) have landed
+        __syncwarp();
+      }
+      const float* sk = ssc + st * 2 * C::RPW;    // Q8: key scales of this warp's rows
+      const float* sv = KEQV ? sk : sk + C::RPW;  // and value scales
       const uint8_t* kt = smem + st * C::STAGE;
-      const uint8_t* vt = KEQV ? kt : kt + kTileBytes;
+      const uint8_t* vt = KEQV ? kt : kt + C::KT;
       const bool full_tile = p0 + TP <= sg.pe;
       auto row_ptr = [&](const uint8_t* base, int r) {
-        return base + static_cast<size_t>((sub + r * SUB) * Hkv + kvh) * D * 2;
+        return base + static_cast<size_t>((sub + r * SUB) * Hkv + kvh) * D * C::ES;
       };
       // ---- logits of this warp's rows, RB rows at a time.  Each step runs
       // over the RB rows before the next starts (loads, norms, rotation,
@@ -450,11 +502,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
         float2 k2[RB][NC][2];
         if (full_tile) {
 #pragma unroll
-          for (int r = 0; r < RB; ++r) load_lane2<NC>(row_ptr(kt, r0 + r), lane, k2[r]);
+          for (int r = 0; r < RB; ++r) load_row(row_ptr(kt, r0 + r), k2[r]);
         } else {
 #pragma unroll
           for (int r = 0; r < RB; ++r) {
-            if (p0 + sub + (r0 + r) * SUB < sg.pe) load_lane2<NC>(row_ptr(kt, r0 + r), lane, k2[r]);
+            if (p0 + sub + (r0 + r) * SUB < sg.pe) load_row(row_ptr(kt, r0 + r), k2[r]);
             else zero_lane2<NC>(k2[r]);
           }
         }
@@ -527,13 +579,15 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
       if (la.qk_norm) {
         // 1/rms of each row: sums of squares through the same butterfly, then
         // each row's factor from the warp scratch
-        const float s2 = transpose_sum<RPW>(ssr, lane);
+        float s2 = transpose_sum<RPW>(ssr, lane);
         const int ri = transpose_index<RPW>(lane);
+        if constexpr (Q8) s2 *= sk[ri] * sk[ri];  // of the dequantised row
         __syncwarp();
         scr[32 + ri] = rsqrtf(s2 / static_cast<float>(D) + la.eps);
         __syncwarp();
         x *= scr[32 + ir];
       }
+      if constexpr (Q8) x *= sk[ir];
       const bool vis = p0 + sub + ir * SUB < sg.pe;
       x = vis ? (cap ? cap_l2 * tanh_fast(x) : x) : -INFINITY;
       // ---- online softmax: tile maxima per head (over the row bits of idx)
@@ -557,7 +611,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
       const float p = vis ? ex2(x - mnew_own) : 0.f;
       lacc = lacc * alpha_own + p;
       __syncwarp();
-      scr[idx] = p;
+      scr[idx] = Q8 ? p * sv[ir] : p;  // P V reads the value scale with the weight
       __syncwarp();
       float pv[NV];
 #pragma unroll
@@ -580,11 +634,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
         float2 v2[RB][NC][2];
         if (full_tile) {
 #pragma unroll
-          for (int r = 0; r < RB; ++r) load_lane2<NC>(row_ptr(vt, r0 + r), lane, v2[r]);
+          for (int r = 0; r < RB; ++r) load_row(row_ptr(vt, r0 + r), v2[r]);
         } else {
 #pragma unroll
           for (int r = 0; r < RB; ++r) {
-            if (p0 + sub + (r0 + r) * SUB < sg.pe) load_lane2<NC>(row_ptr(vt, r0 + r), lane, v2[r]);
+            if (p0 + sub + (r0 + r) * SUB < sg.pe) load_row(row_ptr(vt, r0 + r), v2[r]);
             else zero_lane2<NC>(v2[r]);
           }
         }
@@ -606,6 +660,10 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
         const bool more = ahead.next(P, &tb, &tp0, &tn);  // tile t + NST, if any
         __threadfence_block();  // this warp's reads of the stage are done
         if (lane == 0 && (atomicAdd(&done_cnt[st], 1) % kSW) == kSW - 1 && more) issue(st, tb, tp0, tn);
+        if constexpr (Q8) {
+          if (more) copy_scales(st, tb, tp0, tn);
+          else cp_async_commit();
+        }
       }
     }
     if (!ok) break;
@@ -629,6 +687,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
       }
     }
   }
+  if constexpr (Q8) cp_async_wait<0>();  // no scale copy outlives the CTA
   if (*abort_flag) {
     // after a failed wait, copies issued just before it may still be landing:
     // give them ~100 us before the CTA may exit
@@ -640,9 +699,9 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
 
 namespace {
 
-template <int D, int G, bool KEQV>
+template <int D, int G, bool KEQV, bool Q8>
 cudaError_t run_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
-  using C = SimtShape<D, G, KEQV>;
+  using C = SimtShape<D, G, KEQV, Q8>;
   constexpr int kMaxDev = 64;
   static bool attr_set[kMaxDev] = {};
   int dev = 0, sms = 0;
@@ -650,7 +709,7 @@ cudaError_t run_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStrea
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  auto kern = decode_simt_kernel<D, G, KEQV>;
+  auto kern = decode_simt_kernel<D, G, KEQV, Q8>;
   if (!attr_set[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
@@ -695,35 +754,41 @@ void decode_simt_plan(const LayerArgs& la, int B, int max_len, int max_split, in
   *nsplit = ((span + c - 1) / c) * SUB;
 }
 
-cudaError_t launch_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+template <bool Q8>
+static cudaError_t launch_decode_simt_t(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
   if (la.D == 256) {
     if (la.k_eq_v) {
       switch (la.G) {
-        case 1: return run_decode_simt<256, 1, true>(da, la, s);
-        case 2: return run_decode_simt<256, 2, true>(da, la, s);
-        case 4: return run_decode_simt<256, 4, true>(da, la, s);
+        case 1: return run_decode_simt<256, 1, true, Q8>(da, la, s);
+        case 2: return run_decode_simt<256, 2, true, Q8>(da, la, s);
+        case 4: return run_decode_simt<256, 4, true, Q8>(da, la, s);
       }
     } else {
       switch (la.G) {
-        case 1: return run_decode_simt<256, 1, false>(da, la, s);
-        case 2: return run_decode_simt<256, 2, false>(da, la, s);
-        case 4: return run_decode_simt<256, 4, false>(da, la, s);
+        case 1: return run_decode_simt<256, 1, false, Q8>(da, la, s);
+        case 2: return run_decode_simt<256, 2, false, Q8>(da, la, s);
+        case 4: return run_decode_simt<256, 4, false, Q8>(da, la, s);
       }
     }
   } else if (la.D == 512) {
     if (la.k_eq_v) {
       switch (la.G) {
-        case 1: return run_decode_simt<512, 1, true>(da, la, s);
-        case 2: return run_decode_simt<512, 2, true>(da, la, s);
+        case 1: return run_decode_simt<512, 1, true, Q8>(da, la, s);
+        case 2: return run_decode_simt<512, 2, true, Q8>(da, la, s);
       }
     } else {
       switch (la.G) {
-        case 1: return run_decode_simt<512, 1, false>(da, la, s);
-        case 2: return run_decode_simt<512, 2, false>(da, la, s);
+        case 1: return run_decode_simt<512, 1, false, Q8>(da, la, s);
+        case 2: return run_decode_simt<512, 2, false, Q8>(da, la, s);
       }
     }
   }
   return cudaErrorInvalidValue;
+}
+
+// an int8 cache when da.kq is set, else bf16
+cudaError_t launch_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
+  return da.kq ? launch_decode_simt_t<true>(da, la, s) : launch_decode_simt_t<false>(da, la, s);
 }
 
 }  // namespace gattn

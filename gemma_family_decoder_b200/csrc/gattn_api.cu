@@ -340,6 +340,35 @@ size_t gattn_decode_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t 
          rows * 2 * sizeof(float);
 }
 
+// The split plan, the workspace carve-up and the two launches of a decode call
+// (da holds the cache pointers: bf16 k / v, or int8 kq / vq with their scales).
+static int decode_launch(gattn::DecodeArgs& da, const gattn::LayerArgs& la, const gattn_bf16* q,
+                         const int32_t* seq_lens, gattn_bf16* out, int32_t batch, int32_t max_len,
+                         void* workspace, gattn_stream stream) {
+  gattn::decode_plan(la, batch, max_len, &da.nsplit, &da.chunk);
+  const size_t rows = static_cast<size_t>(batch) * la.H * da.nsplit;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  da.part_o = reinterpret_cast<float*>(ws + round_up(kStatusBytes, 1024));
+  da.part_ml = reinterpret_cast<float*>(ws + round_up(kStatusBytes, 1024) +
+                                        round_up(rows * la.D * sizeof(float), 1024));
+  da.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  da.seq_lens = seq_lens;
+  da.out = reinterpret_cast<__nv_bfloat16*>(out);
+  da.B = batch;
+  da.max_len = max_len;
+  da.status = static_cast<uint32_t*>(workspace);
+  da.trace = static_cast<unsigned long long*>(g_trace_buf);
+  da.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (g_prof_start) cudaEventRecord(g_prof_start, s);
+  cudaError_t e = da.kq ? gattn::launch_decode_simt(da, la, s) : gattn::launch_decode_split(da, la, s);
+  if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
+  if (e != cudaSuccess) return fail_cuda(e, "decode split launch");
+  e = gattn::launch_decode_combine(da, la, s);
+  if (e != cudaSuccess) return fail_cuda(e, "decode combine launch");
+  return GATTN_OK;
+}
+
 int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf16* v_cache_or_null,
                  const int32_t* seq_lens, gattn_bf16* out, int32_t batch, int32_t max_len,
                  const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream) {
@@ -369,30 +398,64 @@ int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf1
   if (batch == 0) return GATTN_OK;
 
   gattn::DecodeArgs da;
-  gattn::decode_plan(la, batch, max_len, &da.nsplit, &da.chunk);
-  const size_t rows = static_cast<size_t>(batch) * la.H * da.nsplit;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  da.part_o = reinterpret_cast<float*>(ws + round_up(kStatusBytes, 1024));
-  da.part_ml = reinterpret_cast<float*>(ws + round_up(kStatusBytes, 1024) +
-                                        round_up(rows * la.D * sizeof(float), 1024));
-  da.q = reinterpret_cast<const __nv_bfloat16*>(q);
   da.k = reinterpret_cast<const __nv_bfloat16*>(k_cache);
   da.v = la.k_eq_v ? da.k : reinterpret_cast<const __nv_bfloat16*>(v_cache_or_null);
-  da.seq_lens = seq_lens;
-  da.out = reinterpret_cast<__nv_bfloat16*>(out);
-  da.B = batch;
-  da.max_len = max_len;
-  da.status = static_cast<uint32_t*>(workspace);
-  da.trace = static_cast<unsigned long long*>(g_trace_buf);
-  da.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (g_prof_start) cudaEventRecord(g_prof_start, s);
-  cudaError_t e = gattn::launch_decode_split(da, la, s);
-  if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
-  if (e != cudaSuccess) return fail_cuda(e, "decode split launch");
-  e = gattn::launch_decode_combine(da, la, s);
-  if (e != cudaSuccess) return fail_cuda(e, "decode combine launch");
+  return decode_launch(da, la, q, seq_lens, out, batch, max_len, workspace, stream);
+}
+
+// ---- int8 KV cache -------------------------------------------------------------------
+int gattn_kv_quantize(const gattn_bf16* x, int8_t* codes, float* scales, int64_t n_rows, int32_t head_dim,
+                      gattn_stream stream) {
+  g_last_error[0] = 0;
+  if (head_dim != 256 && head_dim != 512) return fail(GATTN_ERR_UNSUPPORTED, "head_dim must be 256 or 512");
+  if (n_rows < 0) return fail(GATTN_ERR_INVALID_ARG, "n_rows must be >= 0");
+  if (n_rows == 0) return GATTN_OK;
+  if (!x || !codes || !scales) return fail(GATTN_ERR_INVALID_ARG, "x, codes and scales must not be NULL");
+  if (!aligned16(x) || !aligned16(codes)) return fail(GATTN_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(scales) & 3u) return fail(GATTN_ERR_INVALID_ARG, "scales must be 4-byte aligned");
+  cudaError_t e = gattn::launch_kv_quantize(reinterpret_cast<const __nv_bfloat16*>(x), codes, scales, n_rows,
+                                            head_dim, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "kv quantize launch");
   return GATTN_OK;
+}
+
+int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k_scales,
+                      const int8_t* v_codes_or_null, const float* v_scales_or_null, const int32_t* seq_lens,
+                      gattn_bf16* out, int32_t batch, int32_t max_len, const gattn_cfg* cfg, void* workspace,
+                      size_t ws_bytes, gattn_stream stream) {
+  g_last_error[0] = 0;
+  gattn::LayerArgs la;
+  int st = resolve(cfg, &la, true);
+  if (st != GATTN_OK) return st;
+  if (!gattn::decode_simt_supported(la))
+    return fail(GATTN_ERR_UNSUPPORTED,
+                "int8 cache: 1, 2 or 4 query heads per kv head (head_dim 512: 1 or 2) and 1, 2, 4 or 8 kv heads");
+  if (batch < 0 || max_len <= 0) return fail(GATTN_ERR_INVALID_ARG, "batch must be >= 0 and max_len > 0");
+  if (!q || !k_codes || !k_scales || !out || !seq_lens)
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_codes, k_scales, seq_lens and out must not be NULL");
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(out))
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_codes and out must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(k_scales) & 3u))
+    return fail(GATTN_ERR_INVALID_ARG, "seq_lens and k_scales must be 4-byte aligned");
+  if (la.k_eq_v) {
+    if ((v_codes_or_null && v_codes_or_null != k_codes) || (v_scales_or_null && v_scales_or_null != k_scales))
+      return fail(GATTN_ERR_INVALID_ARG, "k_eq_v: v_codes / v_scales must be NULL or the key arrays");
+  } else {
+    if (!v_codes_or_null || !v_scales_or_null)
+      return fail(GATTN_ERR_INVALID_ARG, "v_codes / v_scales are NULL without k_eq_v");
+    if (!aligned16(v_codes_or_null) || (reinterpret_cast<uintptr_t>(v_scales_or_null) & 3u))
+      return fail(GATTN_ERR_INVALID_ARG, "v_codes must be 16-byte and v_scales 4-byte aligned");
+  }
+  const size_t need = gattn_decode_workspace_size(cfg, batch, max_len);
+  if (!workspace || ws_bytes < need) return fail(GATTN_ERR_WORKSPACE, "workspace missing or too small");
+  if (!aligned16(workspace)) return fail(GATTN_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (batch == 0) return GATTN_OK;
+  gattn::DecodeArgs da;
+  da.kq = k_codes;
+  da.ks = k_scales;
+  da.vq = la.k_eq_v ? k_codes : v_codes_or_null;
+  da.vs = la.k_eq_v ? k_scales : v_scales_or_null;
+  return decode_launch(da, la, q, seq_lens, out, batch, max_len, workspace, stream);
 }
 
 // ---- status ------------------------------------------------------------------------

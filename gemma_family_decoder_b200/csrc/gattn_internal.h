@@ -53,6 +53,11 @@ struct DecodeArgs {
   uint32_t* status;
   unsigned long long* trace = nullptr;  // optional per-CTA timeline (tensor-core kernel)
   size_t trace_bytes = 0;
+  // int8 cache (instead of k / v): codes [B][max_len][Hkv][D], fp32 scales [B][max_len][Hkv]
+  const int8_t* kq = nullptr;
+  const int8_t* vq = nullptr;
+  const float* ks = nullptr;
+  const float* vs = nullptr;
 };
 // Split plan of a decode call: keys per chunk and split slots per (b, head),
 // with at most `max_split` slots (fewer, longer chunks when the plan would
@@ -72,6 +77,9 @@ cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStre
 bool decode_simt_supported(const LayerArgs& la);
 void decode_simt_plan(const LayerArgs& la, int B, int max_len, int max_split, int* nsplit, int* chunk);
 cudaError_t launch_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
+// int8 cache rows: codes and scales of nrows rows of head_dim D (256 or 512)
+cudaError_t launch_kv_quantize(const __nv_bfloat16* x, int8_t* codes, float* scales, long long nrows, int D,
+                               cudaStream_t s);
 
 // Prefill on tcgen05 tensor cores.
 struct PrefillArgs {

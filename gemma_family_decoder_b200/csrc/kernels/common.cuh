@@ -440,4 +440,28 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
+// Four int8 codes (bytes 0..3 of w) as floats, exactly: byte e with its sign
+// bit flipped (code + 128) becomes the low mantissa byte of 2^23, and
+// subtracting 2^23 + 128 leaves the code.  lo = codes 0, 1; hi = codes 2, 3.
+__device__ __forceinline__ void unpack_i8x4(uint32_t w, float2& lo, float2& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float2 off = make_float2(-8388736.f, -8388736.f);
+  lo = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440)),
+                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441))), off);
+  hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442)),
+                              __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443))), off);
+}
+
+// 4-byte asynchronous copies global -> shared, tracked per thread in commit groups
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 }  // namespace gattn

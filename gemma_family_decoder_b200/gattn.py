@@ -27,7 +27,8 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_rope_table_fill", "gattn_workspace_init", "gattn_prefill_workspace_size",
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
-           "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded")
+           "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded", "gattn_kv_quantize",
+           "gattn_decode_int8")
 
 
 class GattnError(RuntimeError):
@@ -100,6 +101,10 @@ def lib() -> ctypes.CDLL:
         L.gattn_set_trace_buffer.argtypes = [vp, sz]
         L.gattn_decode_noalloc.restype = ctypes.c_int
         L.gattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp]
+        L.gattn_kv_quantize.restype = ctypes.c_int
+        L.gattn_kv_quantize.argtypes = [vp, vp, vp, ctypes.c_int64, i32, vp]
+        L.gattn_decode_int8.restype = ctypes.c_int
+        L.gattn_decode_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz, vp]
         L.gattn_prefill_padded.restype = ctypes.c_int
         L.gattn_prefill_padded.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz,
                                            vp]
@@ -248,6 +253,42 @@ class AttentionLayer:
                                      B, Lmax, ctypes.byref(self.cfg), _ptr(ws), ws.numel(),
                                      _stream(stream)), "gattn_decode")
         return out
+
+
+    def decode_int8(self, q, k_codes, k_scales, v_codes=None, v_scales=None, seq_lens=None, out=None,
+                    workspace=None, stream=None):
+        """gattn_decode_int8: q [B,H,D] bf16; codes [B,Lmax,Hkv,D] int8 and scales [B,Lmax,Hkv] fp32
+        (from ``kv_quantize``) of the raw keys/values; seq_lens [B] int32."""
+        _need(q, "q", torch.bfloat16, 3)
+        _need(k_codes, "k_codes", torch.int8, 4)
+        _need(k_scales, "k_scales", torch.float32, 3)
+        if v_codes is not None:
+            _need(v_codes, "v_codes", torch.int8, 4)
+            _need(v_scales, "v_scales", torch.float32, 3)
+        _need(seq_lens, "seq_lens", torch.int32, 1)
+        B, Lmax = k_codes.shape[0], k_codes.shape[1]
+        if tuple(k_scales.shape) != tuple(k_codes.shape[:3]):
+            raise ValueError("k_scales must be [B, Lmax, Hkv]")
+        if v_codes is not None and tuple(v_scales.shape) != tuple(v_codes.shape[:3]):
+            raise ValueError("v_scales must be [B, Lmax, Hkv]")
+        out = torch.empty_like(q) if out is None else out
+        ws = self.decode_workspace(B, Lmax, q.device) if workspace is None else workspace
+        _raise_if(lib().gattn_decode_int8(_ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                          _ptr(seq_lens), _ptr(out), B, Lmax, ctypes.byref(self.cfg), _ptr(ws),
+                                          ws.numel(), _stream(stream)), "gattn_decode_int8")
+        return out
+
+
+def kv_quantize(x: torch.Tensor, codes=None, scales=None, stream=None):
+    """gattn_kv_quantize: x [..., D] bf16 -> (codes [..., D] int8, scales [...] fp32)."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() < 1:
+        raise ValueError("x: expected a contiguous CUDA bfloat16 tensor")
+    D = x.shape[-1]
+    codes = torch.empty(x.shape, dtype=torch.int8, device=x.device) if codes is None else codes
+    scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scales is None else scales
+    _raise_if(lib().gattn_kv_quantize(_ptr(x), _ptr(codes), _ptr(scales), x.numel() // max(D, 1), D,
+                                      _stream(stream)), "gattn_kv_quantize")
+    return codes, scales
 
 
 def decode_noalloc(layer: "AttentionLayer", q, k_cache, v_cache=None, seq_lens=None, out=None,

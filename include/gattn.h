@@ -162,6 +162,38 @@ int gattn_decode(const gattn_bf16* q, const gattn_bf16* k_cache, const gattn_bf1
                  const int32_t* seq_lens, gattn_bf16* out, int32_t batch, int32_t max_len,
                  const gattn_cfg* cfg, void* workspace, size_t ws_bytes, gattn_stream stream);
 
+/* ---- int8 KV cache ------------------------------------------------------------
+ * The Atlas summary of the Gemma 4 report offers int8 KV caching (Table 3, "+KV"
+ * at 32k context) without giving the format.  Here: every cache row (the
+ * head_dim values of one position and one kv head) is stored as int8 codes c and
+ * one fp32 scale s, dequantised as c * s; s = max|x| / 127 and
+ * c = round-half-even(x / s) clipped to [-127, 127], both divisions in IEEE
+ * float32 (a row of zeros: s = 0, codes 0).  Inputs must be finite.
+ *
+ * gattn_kv_quantize: x [n_rows][head_dim] bf16 -> codes [n_rows][head_dim]
+ * int8 and scales [n_rows] fp32 (all device; a [batch][len][Hkv][D] cache is
+ * n_rows = batch * len * Hkv).  head_dim 256 or 512 (else
+ * GATTN_ERR_UNSUPPORTED); x and codes 16-byte aligned, scales 4-byte aligned.
+ * The codes and scales equal a float32 evaluation of the definition bit for bit.
+ * Enqueued on `stream`; no workspace, no status word. */
+int gattn_kv_quantize(const gattn_bf16* x, int8_t* codes, float* scales, int64_t n_rows, int32_t head_dim,
+                      gattn_stream stream);
+
+/* gattn_decode_int8: gattn_decode over an int8 cache, computing with the
+ * dequantised rows (the same RAW keys/values as gattn_decode's caches).
+ *   k_codes / v_codes   [batch][max_len][Hkv][D] int8, 16-byte aligned
+ *   k_scales / v_scales [batch][max_len][Hkv] fp32, 4-byte aligned
+ *   with k_eq_v: v_codes / v_scales NULL (or the key arrays); values are the
+ *   dequantised raw keys.
+ * Every other argument, the workspace size (gattn_decode_workspace_size) and
+ * the errors are those of gattn_decode.  Layers: 1, 2 or 4 query heads per kv
+ * head (head_dim 512: 1 or 2) and 1, 2, 4 or 8 kv heads; others return
+ * GATTN_ERR_UNSUPPORTED. */
+int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k_scales,
+                      const int8_t* v_codes_or_null, const float* v_scales_or_null, const int32_t* seq_lens,
+                      gattn_bf16* out, int32_t batch, int32_t max_len, const gattn_cfg* cfg, void* workspace,
+                      size_t ws_bytes, gattn_stream stream);
+
 /* ---- decode without a workspace ----------------------------------------------------
  * The model cards describe no such call; it exists for callers that cannot
  * allocate device memory at the point where they decode: code running inside

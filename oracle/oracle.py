@@ -296,7 +296,11 @@ def attention_decode_int8(q, k_codes, k_scales, v_codes, v_scales, seq_lens, cfg
     the dequantised raw keys (v_codes / v_scales unused).
     """
     f = _layer_fields(cfg)
-    kd = [kv_dequantize(k_codes[b], k_scales[b]) for b in range(len(k_codes))]
-    vd = None if f["k_eq_v"] else [kv_dequantize(v_codes[b], v_scales[b]) for b in range(len(v_codes))]
+
+    def deq(codes, scales):  # batch rows given as None are left out (see ``batches``)
+        return [None if codes[b] is None else kv_dequantize(codes[b], scales[b]) for b in range(len(codes))]
+
+    kd = deq(k_codes, k_scales)
+    vd = None if f["k_eq_v"] else deq(v_codes, v_scales)
     return attention_decode(q, kd, vd, seq_lens, cfg, w_q=w_q, w_k=w_k, batches=batches,
                             first_rows=first_rows)

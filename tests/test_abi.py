@@ -108,6 +108,35 @@ def test_prefill_padded_rejects_bad_args():
     assert G.lib().gattn_last_error() == b""
 
 
+def test_kv_quantize_rejects_bad_args():
+    L = G.lib()
+    assert L.gattn_kv_quantize(ALIGNED, ALIGNED, ALIGNED, 4, 128, None) == UNSUPPORTED
+    assert L.gattn_kv_quantize(ALIGNED, ALIGNED, ALIGNED, -1, 256, None) == INVALID
+    assert L.gattn_kv_quantize(None, ALIGNED, ALIGNED, 4, 256, None) == INVALID
+    assert L.gattn_kv_quantize(ALIGNED + 8, ALIGNED, ALIGNED, 4, 256, None) == INVALID
+    assert L.gattn_kv_quantize(ALIGNED, ALIGNED, ALIGNED + 2, 4, 256, None) == INVALID
+    assert L.gattn_kv_quantize(ALIGNED, ALIGNED, ALIGNED, 0, 256, None) == 0   # nothing to do
+
+
+def decode_int8(c, q=ALIGNED, kc=ALIGNED, ks=ALIGNED, vc=ALIGNED, vs=ALIGNED, lens=ALIGNED, out=ALIGNED, B=1,
+                Lmax=16, ws=ALIGNED, ws_bytes=1 << 30):
+    return G.lib().gattn_decode_int8(q, kc, ks, vc, vs, lens, out, B, Lmax, ctypes.byref(c), ws, ws_bytes, None)
+
+
+def test_decode_int8_rejects_bad_args():
+    c = cfg(num_heads=16, num_kv_heads=8)
+    assert decode_int8(cfg(num_heads=16, num_kv_heads=1)) == UNSUPPORTED   # 16 per kv head: no int8 kernel
+    assert decode_int8(c, kc=None) == INVALID
+    assert decode_int8(c, ks=ALIGNED + 2) == INVALID
+    assert decode_int8(c, kc=ALIGNED + 4) == INVALID
+    assert decode_int8(c, vs=None) == INVALID                              # separate values need scales
+    ck = cfg(num_heads=4, num_kv_heads=2, k_eq_v=1)
+    assert decode_int8(ck, vc=ALIGNED + 4096, vs=None) == INVALID         # tied: v arrays NULL or the key ones
+    assert decode_int8(ck, vc=None, vs=None, B=0) == 0
+    assert decode_int8(c, ws_bytes=16) == WORKSPACE
+    assert decode_int8(c, B=0) == 0
+
+
 def test_empty_problem_is_a_no_op():
     assert prefill(cfg(), B=0) == 0
     assert prefill(cfg(), S=0) == 0

@@ -82,7 +82,7 @@ MUTATIONS = {
         [T8.test_round_trip_within_half_step_and_extremes,
          T8.test_int8_decode_equals_float_decode_on_representable_cache]),
     "int8_values_from_key_codes": (
-        "[kv_dequantize(v_codes[b], v_scales[b])", "[kv_dequantize(k_codes[b], v_scales[b])",
+        "else deq(v_codes, v_scales)", "else deq(k_codes, v_scales)",
         [T8.test_int8_decode_equals_float_decode_on_representable_cache]),
 }
 

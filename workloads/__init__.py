@@ -85,6 +85,9 @@ class DecodeWorkload:
     seed: int
     gain_mean: float = 0.0
     gain_std: float = 0.1
+    # the cache held as int8 codes + fp32 row scales (Atlas "Gemma 4" summary: int8 KV
+    # caching), quantised from the same bf16 rows
+    kv_int8: bool = False
 
     @property
     def max_len(self) -> int:
@@ -145,10 +148,14 @@ GEMMA3_GLOBAL_LEFTPAD = PrefillWorkload(
     "gemma3_1b_global_b8_s4096_leftpad",
     Layer(window=0, rope_theta=1e6, **_G3), batch=8, seq=4096, seed=5, len_lo=512)
 
+# the local decode layer over an int8 cache of the same rows
+GEMMA4_DECODE_LOCAL_INT8 = dataclasses.replace(GEMMA4_DECODE_LOCAL, name="gemma4_12b_decode_local_int8_b64",
+                                               kv_int8=True)
+
 PREFILL: Dict[str, PrefillWorkload] = {w.name: w for w in (
     GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL, GEMMA3_GLOBAL_LEFTPAD)}
 DECODE: Dict[str, DecodeWorkload] = {w.name: w for w in (
-    GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM)}
+    GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM, GEMMA4_DECODE_LOCAL_INT8)}
 
 
 # --- drawing -------------------------------------------------------------------
