@@ -14,6 +14,7 @@ import oracle
 import oracle.oracle as src_mod
 import test_oracle as T
 import test_oracle_int8 as T8
+import test_oracle_chunk as TC
 
 MUTATIONS = {
     # name: (original text, replacement, pins that must fail)
@@ -81,6 +82,13 @@ MUTATIONS = {
         "return np.asarray(codes, dtype=np.float64)",
         [T8.test_round_trip_within_half_step_and_extremes,
          T8.test_int8_decode_equals_float_decode_on_representable_cache]),
+    "chunk_queries_at_local_positions": (
+        "q_idx = P + np.arange(C)                    # chunk token i: token P + i",
+        "q_idx = np.arange(C)",
+        [TC.test_chunk_equals_rows_of_whole_prompt, TC.test_chunk_onehot_counts]),
+    "chunk_sees_only_prefix": (
+        "n = P + C                                   # cache rows the chunk can see", "n = max(P, 1)",
+        [TC.test_chunk_equals_rows_of_whole_prompt]),
     "int8_values_from_key_codes": (
         "else deq(v_codes, v_scales)", "else deq(k_codes, v_scales)",
         [T8.test_int8_decode_equals_float_decode_on_representable_cache]),
