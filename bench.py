@@ -47,6 +47,7 @@ PREFILL_WL = {
 }
 DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
                                  W.GEMMA4_DECODE_GLOBAL_NORM, W.GEMMA4_DECODE_LOCAL_INT8)}
+CHUNK_WL = {W.GEMMA3_GLOBAL_CHUNK.name: W.GEMMA3_GLOBAL_CHUNK}
 HEADLINE = "gemma1_2b_mqa_b4_s2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -73,6 +74,13 @@ def prefill_flops(wl: W.PrefillWorkload, seq_range=None) -> float:
         return 4.0 * L.head_dim * L.num_heads * wl.batch * visible_pairs(wl.seq, L.window)
     pairs = sum(visible_pairs(int(hi) - int(lo), L.window) for lo, hi in seq_range.tolist() if hi > lo)
     return 4.0 * L.head_dim * L.num_heads * pairs
+
+
+def chunk_flops(wl: W.ChunkWorkload, rows=None) -> float:
+    """Q K^T and P V FLOPs of the chunk rows ``rows`` (default all): row i is token prefix + i."""
+    L = wl.layer
+    rows = np.arange(wl.chunk) if rows is None else np.asarray(rows, dtype=np.int64)
+    return 4.0 * L.head_dim * L.num_heads * wl.batch * float(row_visible(wl.prefix + rows, L.window).sum())
 
 
 def rows_flops(wl: W.PrefillWorkload, d, rows) -> float:
@@ -249,6 +257,32 @@ def make_prefill(wl, dev):
                 oracle=lambda: d)
 
 
+def make_chunk(wl, dev):
+    from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
+    d = W.chunk_inputs(wl)
+    layer = AttentionLayer(LayerSpec.of(wl.layer), d["max_len"], d["w_q"], d["w_k"], device=dev)
+    host = {k: d[k].pin_memory() for k in ("q", "k_new", "v_new", "prefix_lens") if d[k] is not None}
+    devt = {k: t.to(dev) for k, t in host.items()}
+    k_cache = d["k_cache"].to(dev)
+    v_cache = None if d["v_cache"] is None else d["v_cache"].to(dev)
+    out = torch.empty_like(devt["q"])
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    ws = layer.prefill_chunk_workspace(wl.batch, wl.chunk, d["max_len"], dev)
+
+    def step(src=devt):
+        # append the chunk's rows to the cache, then attend (rewriting the same rows every step)
+        layer.prefill_chunk(src["q"], k_cache, v_cache, src["prefix_lens"], k_new=src["k_new"], v_new=src.get("v_new"),
+                            out=out, workspace=ws)
+
+    prep = bool(wl.layer.rot_dim or wl.layer.qk_norm)
+    return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
+                work=chunk_flops(wl), unit="TFLOP/s", scale=1e12,
+                metric="attention prefill TFLOP/s (effective FLOPs)", bound="tensor",
+                launches=4 if prep else 2,
+                kernel_src=("gemma_family_decoder_b200/csrc/prefill.cu",
+                            "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
+
+
 def make_decode(wl, dev):
     from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
     dq = W.decode_inputs(wl)
@@ -300,12 +334,13 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     name = args.workload
     is_prefill = name in PREFILL_WL
-    wl = PREFILL_WL[name] if is_prefill else DECODE_WL[name]
-    if args.len_hi and not is_prefill:
+    is_chunk = name in CHUNK_WL
+    wl = PREFILL_WL[name] if is_prefill else CHUNK_WL[name] if is_chunk else DECODE_WL[name]
+    if args.len_hi and not is_prefill and not is_chunk:
         # a smaller cache for profiling; with a window no longer than the
         # shortest sequence the work per step is the same
         wl = dataclasses.replace(wl, len_hi=max(wl.len_lo, args.len_hi))
-    R = make_prefill(wl, dev) if is_prefill else make_decode(wl, dev)
+    R = make_prefill(wl, dev) if is_prefill else make_chunk(wl, dev) if is_chunk else make_decode(wl, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     flush_r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -413,7 +448,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": name, "l2": "flushed before every step (256 MiB write, then a 256 MiB read "
                    "that drains the write's dirty lines), outside the per-step CUDA-event time",
                    "step": "eager library call" if graph is None else "CUDA-graph replay of the library call",
-                   **({"len_hi": wl.len_hi} if args.len_hi and not is_prefill else {}),
+                   **({"len_hi": wl.len_hi} if args.len_hi and not is_prefill and not is_chunk else {}),
                    "parallelism": f"replicas{world}"},
         "roofline": {"bound": R["bound"], "achieved": round(achieved, 3), "peak": peak,
                      "unit": peak_unit, "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -464,9 +499,40 @@ def _oracle_decode(wl, dq, cache, batches, firsts):
                               w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts)
 
 
+def _oracle_chunk(wl, d, rows):
+    import oracle as O
+    kc = d["k_cache"].clone()
+    kc[:, wl.prefix:] = d["k_new"]
+    vc = None
+    if d["v_cache"] is not None:
+        vc = d["v_cache"].clone()
+        vc[:, wl.prefix:] = d["v_new"]
+    return O.attention_prefill_chunk(d["q"], kc, vc, d["prefix_lens"], wl.layer, w_q=d["w_q"], w_k=d["w_k"],
+                                     rows=rows)
+
+
 def cpu_baseline(name, budget_s=15.0):
     """The oracle timed on a strided sample of query rows (prefill) or batch rows (decode)."""
     import oracle as O
+    if name in CHUNK_WL:
+        wl = CHUNK_WL[name]
+        d = W.chunk_inputs(wl)
+        _oracle_chunk(wl, d, np.array([0]))  # warm-up
+        # rows cost little next to each call's key transform: grow the strided sample
+        # until it takes about a quarter of the budget (or is the whole chunk)
+        n = 16
+        while True:
+            rows = np.unique(np.linspace(0, wl.chunk - 1, n).astype(np.int64))
+            t0 = time.perf_counter()
+            _oracle_chunk(wl, d, rows)
+            dt = time.perf_counter() - t0
+            if n >= wl.chunk or dt > budget_s / 4:
+                break
+            n = min(wl.chunk, n * 4)
+        return {"value": round(chunk_flops(wl, rows) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+                "kind": "oracle",
+                "sample": f"{len(rows)} evenly spaced chunk rows of {wl.chunk}, all {wl.batch} sequences and "
+                          f"{wl.layer.num_heads} heads ({dt:.1f} s, float64 numpy)"}
     if name in PREFILL_WL:
         wl = PREFILL_WL[name]
         d = W.prefill_inputs(wl)
@@ -520,7 +586,27 @@ def run_reference(args, world, rank):
     name = args.workload
     budget = float(os.environ.get("GATTN_REF_BUDGET_S", "120"))
     n_steps = args.steps + args.warmup
-    if name in PREFILL_WL:
+    if name in CHUNK_WL:
+        wl = CHUNK_WL[name]
+        d = W.chunk_inputs(wl)
+        t0 = time.perf_counter()
+        _oracle_chunk(wl, d, np.array([wl.chunk - 1]))
+        per_row = time.perf_counter() - t0
+        rows_per_step = int(max(1, min(wl.chunk, budget / n_steps / max(per_row, 1e-6))))
+        rng = np.random.default_rng(0)
+        work, dt = 0.0, 0.0
+        for i in range(n_steps):
+            rows = np.sort(rng.choice(wl.chunk, size=rows_per_step, replace=False))
+            t0 = time.perf_counter()
+            _oracle_chunk(wl, d, rows)
+            el = time.perf_counter() - t0
+            if i >= args.warmup:
+                dt += el
+                work += chunk_flops(wl, rows)
+        value, unit = work / dt / 1e12, "TFLOP/s"
+        sample = f"{rows_per_step} random chunk rows of {wl.chunk} per step, all sequences and heads"
+        metric = "attention prefill TFLOP/s (effective FLOPs)"
+    elif name in PREFILL_WL:
         wl = PREFILL_WL[name]
         d = W.prefill_inputs(wl)
         S, L = wl.seq, wl.layer
@@ -583,7 +669,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default=HEADLINE, choices=sorted(PREFILL_WL) + sorted(DECODE_WL))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(PREFILL_WL) + sorted(CHUNK_WL) + sorted(DECODE_WL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager library calls instead of a graph replay")
     ap.add_argument("--len-hi", type=int, default=0,

@@ -322,6 +322,121 @@ static int prefill_impl(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf
   return GATTN_OK;
 }
 
+// ---- a chunk against a cached prefix ----------------------------------------------
+size_t gattn_prefill_chunk_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t chunk_len, int32_t max_len) {
+  gattn::LayerArgs la;
+  if (resolve(cfg, &la, false) != GATTN_OK || batch < 0 || chunk_len < 0 || max_len < chunk_len) return 0;
+  size_t bytes = kStatusBytes;
+  if (prefill_needs_kprep(la))  // transformed cache keys, then the chunk's transformed queries
+    bytes = round_up(bytes, 1024) +
+            round_up(static_cast<size_t>(batch) * max_len * la.Hkv * la.D * sizeof(uint16_t), 1024) +
+            static_cast<size_t>(batch) * chunk_len * la.H * la.D * sizeof(uint16_t);
+  return bytes;
+}
+
+int gattn_kv_append(const gattn_bf16* k_new, const gattn_bf16* v_new_or_null, gattn_bf16* k_cache,
+                    gattn_bf16* v_cache_or_null, const int32_t* cache_lens, int32_t batch, int32_t n_new,
+                    int32_t max_len, int32_t num_kv_heads, int32_t head_dim, void* status_or_null,
+                    gattn_stream stream) {
+  g_last_error[0] = 0;
+  if (batch < 0 || n_new < 0 || max_len < n_new || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8)
+    return fail(GATTN_ERR_INVALID_ARG, "need batch, n_new >= 0, max_len >= n_new, num_kv_heads > 0, head_dim % 8 == 0");
+  if (batch == 0 || n_new == 0) return GATTN_OK;
+  if (!k_new || !k_cache || !cache_lens) return fail(GATTN_ERR_INVALID_ARG, "k_new, k_cache and cache_lens must not be NULL");
+  if ((v_new_or_null == nullptr) != (v_cache_or_null == nullptr))
+    return fail(GATTN_ERR_INVALID_ARG, "v_new and v_cache must both be given or both be NULL");
+  if (!aligned16(k_new) || !aligned16(k_cache) || (v_new_or_null && (!aligned16(v_new_or_null) ||
+                                                                    !aligned16(v_cache_or_null))))
+    return fail(GATTN_ERR_INVALID_ARG, "rows must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(cache_lens) & 3u) return fail(GATTN_ERR_INVALID_ARG, "cache_lens must be 4-byte aligned");
+  if (status_or_null && !aligned16(status_or_null)) return fail(GATTN_ERR_INVALID_ARG, "status must be 16-byte aligned");
+  cudaError_t e = gattn::launch_kv_append(
+      reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new_or_null),
+      reinterpret_cast<__nv_bfloat16*>(k_cache), reinterpret_cast<__nv_bfloat16*>(v_cache_or_null), cache_lens, batch,
+      n_new, max_len, num_kv_heads, head_dim, static_cast<uint32_t*>(status_or_null),
+      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "kv append launch");
+  return GATTN_OK;
+}
+
+int gattn_prefill_chunk(const gattn_bf16* q, const gattn_bf16* k_new_or_null, const gattn_bf16* v_new_or_null,
+                        gattn_bf16* k_cache, gattn_bf16* v_cache_or_null, const int32_t* prefix_lens,
+                        gattn_bf16* out, int32_t batch, int32_t chunk_len, int32_t max_len, const gattn_cfg* cfg,
+                        void* workspace, size_t ws_bytes, gattn_stream stream) {
+  g_last_error[0] = 0;
+  gattn::LayerArgs la;
+  int st = resolve(cfg, &la, true);
+  if (st != GATTN_OK) return st;
+  if (batch < 0 || chunk_len < 0 || max_len < chunk_len || max_len <= 0)
+    return fail(GATTN_ERR_INVALID_ARG, "need batch, chunk_len >= 0 and max_len >= max(chunk_len, 1)");
+  if (static_cast<long long>(batch) * max_len * la.H > (1LL << 31) - 1)
+    return fail(GATTN_ERR_INVALID_ARG, "problem too large");
+  if (!q || !k_cache || !out || !prefix_lens)
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_cache, prefix_lens and out must not be NULL");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(out))
+    return fail(GATTN_ERR_INVALID_ARG, "q, k_cache and out must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(prefix_lens) & 3u)
+    return fail(GATTN_ERR_INVALID_ARG, "prefix_lens must be 4-byte aligned");
+  if (la.k_eq_v) {
+    if ((v_cache_or_null && v_cache_or_null != k_cache) || (v_new_or_null && v_new_or_null != k_new_or_null))
+      return fail(GATTN_ERR_INVALID_ARG, "k_eq_v: v_cache / v_new must be NULL or the key arrays");
+  } else {
+    if (!v_cache_or_null) return fail(GATTN_ERR_INVALID_ARG, "v_cache is NULL without k_eq_v");
+    if (!aligned16(v_cache_or_null)) return fail(GATTN_ERR_INVALID_ARG, "v_cache must be 16-byte aligned");
+    if ((k_new_or_null == nullptr) != (v_new_or_null == nullptr))
+      return fail(GATTN_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  }
+  if ((k_new_or_null && !aligned16(k_new_or_null)) || (v_new_or_null && !aligned16(v_new_or_null)))
+    return fail(GATTN_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  const size_t need = gattn_prefill_chunk_workspace_size(cfg, batch, chunk_len, max_len);
+  if (!workspace || ws_bytes < need) return fail(GATTN_ERR_WORKSPACE, "workspace missing or too small");
+  if (!aligned16(workspace)) return fail(GATTN_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (batch == 0 || chunk_len == 0) return GATTN_OK;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
+  __nv_bfloat16* vc = la.k_eq_v ? kc : reinterpret_cast<__nv_bfloat16*>(v_cache_or_null);
+  if (k_new_or_null) {
+    cudaError_t e = gattn::launch_kv_append(
+        reinterpret_cast<const __nv_bfloat16*>(k_new_or_null),
+        la.k_eq_v ? nullptr : reinterpret_cast<const __nv_bfloat16*>(v_new_or_null), kc, la.k_eq_v ? nullptr : vc,
+        prefix_lens, batch, chunk_len, max_len, la.Hkv, la.D, status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "kv append launch");
+  }
+  const __nv_bfloat16* kt = kc;
+  const __nv_bfloat16* qt = reinterpret_cast<const __nv_bfloat16*>(q);
+  if (prefill_needs_kprep(la)) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    __nv_bfloat16* ktw = reinterpret_cast<__nv_bfloat16*>(ws + round_up(kStatusBytes, 1024));
+    __nv_bfloat16* qtw = reinterpret_cast<__nv_bfloat16*>(
+        ws + round_up(kStatusBytes, 1024) +
+        round_up(static_cast<size_t>(batch) * max_len * la.Hkv * la.D * sizeof(uint16_t), 1024));
+    cudaError_t e = gattn::launch_qkprep_chunk(qt, kc, prefix_lens, qtw, ktw, batch, chunk_len, max_len, la, status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "query/key prologue launch");
+    kt = ktw;
+    qt = qtw;
+  }
+  gattn::PrefillArgs pa;
+  pa.q = qt;
+  pa.kt = kt;
+  pa.v = vc;
+  pa.out = reinterpret_cast<__nv_bfloat16*>(out);
+  pa.B = batch;
+  pa.S = chunk_len;
+  pa.KV_S = max_len;
+  pa.q_off = prefix_lens;
+  pa.status = status;
+  pa.timeout_ns = gattn::wait_timeout_ns();
+  pa.trace = static_cast<unsigned long long*>(g_trace_buf);
+  pa.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
+  if (g_prof_start) cudaEventRecord(g_prof_start, s);
+  cudaError_t e = gattn::launch_prefill(pa, la, s);
+  if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
+  if (e != cudaSuccess) return fail_cuda(e, "chunk prefill launch");
+  return GATTN_OK;
+}
+
 // ---- decode ------------------------------------------------------------------------
 static int decode_supported(const gattn::LayerArgs& la) {
   const int G = la.G;

@@ -35,6 +35,17 @@ cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim,
 
 // q~ = RoPE(RMSNorm(q)) for every (b, s, head) row and k~ = RoPE(RMSNorm(k))
 // for every (b, s, kv head) row, bf16 out, same layouts, in one launch.
+// The chunk form: queries of a chunk (token prefix[b] + i, q only) into qt, and cache
+// keys (token j, rows j < prefix[b] + C only) into kt.
+cudaError_t launch_qkprep_chunk(const __nv_bfloat16* q, const __nv_bfloat16* k_cache, const int* prefix,
+                                __nv_bfloat16* qt, __nv_bfloat16* kt, int B, int C, int max_len,
+                                const LayerArgs& la, uint32_t* status, cudaStream_t s);
+// Copy a chunk's new rows [B][C][Hkv][D] into cache rows [prefix[b], prefix[b] + C)
+// (v_new / v_cache null when keys and values are tied); a prefix outside
+// [0, max_len - C] is clamped and flagged.
+cudaError_t launch_kv_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new, __nv_bfloat16* k_cache,
+                             __nv_bfloat16* v_cache, const int* prefix, int B, int C, int max_len, int Hkv,
+                             int D, uint32_t* status, cudaStream_t s);
 cudaError_t launch_qkprep(const __nv_bfloat16* q, const __nv_bfloat16* k, const int* positions,
                           __nv_bfloat16* qt, __nv_bfloat16* kt, int B, int S, const LayerArgs& la,
                           uint32_t* status, cudaStream_t s);
@@ -93,6 +104,10 @@ struct PrefillArgs {
   unsigned long long* trace;  // optional kernel timeline buffer (null = off)
   size_t trace_bytes;
   const int* seq_range = nullptr;  // [B][2] valid tokens of each sequence (padded batch), or null
+  // a chunk against a cached prefix: query row i of sequence b is token q_off[b] + i; the
+  // keys and values have KV_S rows (the cache), q and out S rows
+  const int* q_off = nullptr;
+  int KV_S = 0;
 };
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
 

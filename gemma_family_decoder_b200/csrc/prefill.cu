@@ -75,6 +75,8 @@ struct PrefillKParams {
   unsigned long long* trace;  // optional per-CTA event times (kTraceSlots each), or null
   int trace_ctas;
   const int* seq_range;       // [B][2] valid tokens [lo, hi) of each sequence, or null (all valid)
+  const int* q_off;           // chunk: token index of each sequence's first query row
+  int KV_S;                   // chunk: key/value rows (the cache length)
 };
 
 // Optional timeline of one CTA's first item (debug aid, off unless a trace
@@ -87,11 +89,14 @@ constexpr int kTraceSlots = 512;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// PAD: the batch is padded (P.seq_range set); a separate instance so that the
-// unpadded kernel carries none of the extra masking
-template <int D, int BN, bool CAP, bool PAD>
+// MODE 0: a whole prompt; 1: a padded batch (P.seq_range); 2: a chunk of S
+// queries against a cache of KV_S rows, query row i of sequence b being token
+// q_off[b] + i.  Separate instances, so the plain kernel carries none of the
+// extra index arithmetic.
+template <int D, int BN, bool CAP, int MODE>
 __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__ PrefillKParams P) {
   using C = PrefillShape<D, BN>;
+  constexpr bool PAD = MODE == 1, CHUNK = MODE == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
@@ -118,6 +123,7 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   struct Item {
     int qt, dvs, h, b, kvh, q0, dv_lo, k_first, ntiles, rot;
     int lo, hi;  // the sequence's valid tokens (all of [0, S) unless the batch is padded)
+    int qa;      // token index of the tile's first row (q0 unless a chunk)
   };
   auto item_of = [&](int it) {
     Item w;
@@ -133,14 +139,21 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
     w.dv_lo = w.dvs * C::DV;
     w.lo = 0;
     w.hi = S;
+    w.qa = w.q0;
     if constexpr (PAD) {
       w.lo = min(max(__ldg(P.seq_range + 2 * w.b), 0), S);
       w.hi = min(max(__ldg(P.seq_range + 2 * w.b + 1), 0), S);
     }
+    if constexpr (CHUNK) {
+      // the chunk's tokens [off, off + S) of a cache of KV_S rows
+      const int off = min(max(__ldg(P.q_off + w.b), 0), P.KV_S - S);
+      w.qa = w.q0 + off;
+      w.hi = off + S;
+    }
     // keys of the tile's valid rows: from the window's (and the sequence's)
     // first key to the last valid row
-    const int kv_hi = min(min(S, w.q0 + C::BM), w.hi);
-    const int kv_lo = max(la.window > 0 ? max(0, w.q0 - la.window + 1) : 0, w.lo);
+    const int kv_hi = min(min(CHUNK ? w.hi : S, w.qa + C::BM), w.hi);
+    const int kv_lo = max(la.window > 0 ? max(0, w.qa - la.window + 1) : 0, w.lo);
     w.k_first = (kv_lo / BN) * BN;
     // a query tile with no valid row reads no keys: its rows are zero
     const bool none = PAD && (w.lo >= w.hi || w.q0 + C::BM <= w.lo || w.q0 >= w.hi);
@@ -227,9 +240,14 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
       const int qi = w.q0 + t;
       const bool in_seq = qi < S;                            // a row of the output
       const bool valid = in_seq && (!PAD || (qi >= w.lo && qi < w.hi));  // and not padding
+      const int qa = w.qa + t;                               // its token index
       if (PAD && t == 0 && w.qt == 0 && w.h == 0 && w.dvs == 0) {
         const int lo_in = __ldg(P.seq_range + 2 * w.b), hi_in = __ldg(P.seq_range + 2 * w.b + 1);
         if (lo_in < 0 || hi_in > S) flag_status(P.status, kStatusBounds);
+      }
+      if (CHUNK && t == 0 && w.qt == 0 && w.h == 0 && w.dvs == 0) {
+        const int off_in = __ldg(P.q_off + w.b);
+        if (off_in < 0 || off_in > P.KV_S - S) flag_status(P.status, kStatusBounds);
       }
       if (PAD && w.ntiles == 0) {
         // every row of the tile is padding: zero output, no keys, no MMAs
@@ -253,9 +271,9 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
         tmem_wait_ld();
 
         const int key0 = tile_key(w, j);
-        const bool full_tile = (key0 + BN - 1 <= w.q0) && (w.q0 + C::BM <= (PAD ? min(S, w.hi) : S)) &&
+        const bool full_tile = (key0 + BN - 1 <= w.qa) && (w.q0 + C::BM <= (PAD ? min(S, w.hi) : S)) &&
                                (!PAD || (key0 >= w.lo && w.q0 >= w.lo)) &&
-                               (W <= 0 || (w.q0 + C::BM - 1) - key0 < W);
+                               (W <= 0 || (w.qa + C::BM - 1) - key0 < W);
         float x[BN];
 #pragma unroll
         for (int i = 0; i < BN; ++i) {
@@ -263,8 +281,8 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
           x[i] = CAP ? cap_l2 * tanh_fast(sv * kcap) : sv;
         }
         if (!full_tile) {
-          const int hi = valid ? qi - key0 : -1;            // visible iff i <= hi
-          const int lo_w = W > 0 ? qi - key0 - W + 1 : -BN;   // and i >= lo
+          const int hi = valid ? qa - key0 : -1;            // visible iff i <= hi
+          const int lo_w = W > 0 ? qa - key0 - W + 1 : -BN;   // and i >= lo
           const int lo = PAD ? max(lo_w, w.lo - key0) : lo_w;
 #pragma unroll
           for (int i = 0; i < BN; ++i) x[i] = (i <= hi && i >= lo) ? x[i] : -INFINITY;
@@ -513,13 +531,14 @@ __global__ void __launch_bounds__(192, 1) prefill_kernel(const __grid_constant__
   if (threadIdx.x == 0) mark(5);
 }
 
-template <int D, int BN, bool CAP, bool PAD>
+template <int D, int BN, bool CAP, int MODE>
 static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   using C = PrefillShape<D, BN>;
   PrefillKParams P;
+  const int kv_rows = MODE == 2 ? pa.KV_S : pa.S;
   if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, D, C::BM) ||
-      !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, D, BN) ||
-      !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, pa.S, la.Hkv, D, BN))
+      !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, kv_rows, la.Hkv, D, BN) ||
+      !encode_tmap_bshd(&P.tm_v, pa.v, pa.B, kv_rows, la.Hkv, D, BN))
     return cudaErrorInvalidValue;
   P.out = pa.out;
   P.status = pa.status;
@@ -532,7 +551,9 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.trace = pa.trace;
   P.trace_ctas = static_cast<int>(pa.trace_bytes / (kTraceSlots * sizeof(unsigned long long)));
   P.seq_range = pa.seq_range;
-  auto kern = prefill_kernel<D, BN, CAP, PAD>;
+  P.q_off = pa.q_off;
+  P.KV_S = kv_rows;
+  auto kern = prefill_kernel<D, BN, CAP, MODE>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -550,20 +571,20 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(192), C::SMEM, s, P);
 }
 
-cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+template <int MODE>
+static cudaError_t launch_prefill_mode(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   const bool cap = la.softcap > 0.f;
-  if (pa.seq_range) {
-    if (la.D == 256)
-      return cap ? run_prefill<256, 128, true, true>(pa, la, s) : run_prefill<256, 128, false, true>(pa, la, s);
-    if (la.D == 512)
-      return cap ? run_prefill<512, 64, true, true>(pa, la, s) : run_prefill<512, 64, false, true>(pa, la, s);
-    return cudaErrorInvalidValue;
-  }
   if (la.D == 256)
-    return cap ? run_prefill<256, 128, true, false>(pa, la, s) : run_prefill<256, 128, false, false>(pa, la, s);
+    return cap ? run_prefill<256, 128, true, MODE>(pa, la, s) : run_prefill<256, 128, false, MODE>(pa, la, s);
   if (la.D == 512)
-    return cap ? run_prefill<512, 64, true, false>(pa, la, s) : run_prefill<512, 64, false, false>(pa, la, s);
+    return cap ? run_prefill<512, 64, true, MODE>(pa, la, s) : run_prefill<512, 64, false, MODE>(pa, la, s);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+  if (pa.seq_range) return launch_prefill_mode<1>(pa, la, s);
+  if (pa.q_off) return launch_prefill_mode<2>(pa, la, s);
+  return launch_prefill_mode<0>(pa, la, s);
 }
 
 }  // namespace gattn

@@ -53,17 +53,37 @@ cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim,
 // rows (query gain) and Hkv key rows (key gain), RB rows at a time with
 // their loads issued together; outputs keep the input layouts.
 // ---------------------------------------------------------------------------
-template <int TPR, int RB>
+// MODE 0: a prompt's queries and keys, positions from `positions`.  MODE 1: a
+// chunk's queries only (token bs = b * C + s at position prefix[b] + s).
+// MODE 2: a cache's keys only (token bs = b * max_len + s at position s),
+// skipping the rows past the chunk (s >= prefix[b] + C).
+struct ChunkPrep {
+  const int* prefix;
+  int C, max_len;
+};
+
+template <int TPR, int RB, int MODE>
 __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                                                      const int* __restrict__ positions,
                                                      bf16* __restrict__ qt, bf16* __restrict__ kt,
-                                                     long long tokens, LayerArgs la, uint32_t* status) {
+                                                     long long tokens, LayerArgs la, uint32_t* status,
+                                                     ChunkPrep cp) {
   constexpr int D = TPR * 16;
   pdl_launch_dependents();  // the attention kernel may be scheduled now; it waits for this grid
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long bs = gid / TPR;
   const int i = static_cast<int>(gid % TPR);
   if (bs >= tokens) return;  // whole groups leave together (TPR divides 32)
+  int tok_pos = 0;
+  if constexpr (MODE == 0) {
+    tok_pos = positions ? __ldg(positions + bs) : 0;
+  } else {
+    const int per = MODE == 1 ? cp.C : cp.max_len;
+    const int b = static_cast<int>(bs / per), s = static_cast<int>(bs % per);
+    const int pre = min(max(__ldg(cp.prefix + b), 0), cp.max_len - cp.C);
+    if (MODE == 2 && s >= pre + cp.C) return;  // a cache row no query of the chunk sees
+    tok_pos = MODE == 1 ? pre + s : s;
+  }
   const unsigned gmask = TPR == 32 ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
   const int h8 = la.rot >> 4;  // chunks in half the rotated slice
   const bool rotated = i < h8;
@@ -71,13 +91,14 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
   const int c1 = rotated ? i + h8 : c0 + 1;
   float4 cs[4];  // (cos, sin) of pairs 8i .. 8i+7, two pairs per float4
   if (rotated) {
-    const int pos = checked_pos(positions ? __ldg(positions + bs) : 0, la, status);
+    const int pos = checked_pos(tok_pos, la, status);
     const float4* trow = reinterpret_cast<const float4*>(la.rope_tab + static_cast<size_t>(pos) * (la.rot >> 1)) + 4 * i;
 #pragma unroll
     for (int e = 0; e < 4; ++e) cs[e] = __ldg(trow + e);
   }
   const float off = la.qk_norm == 1 ? 1.f : 0.f;
-  const int nrows = la.H + la.Hkv;
+  const int nq = MODE == 2 ? 0 : la.H;  // query rows of the token, then key rows
+  const int nrows = nq + (MODE == 1 ? 0 : la.Hkv);
   for (int r0 = 0; r0 < nrows; r0 += RB) {
     uint4 u0[RB], u1[RB];
 #pragma unroll
@@ -85,7 +106,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
       const int r = r0 + u;
       if (r < nrows) {
         const uint4* src = reinterpret_cast<const uint4*>(
-            r < la.H ? q + (bs * la.H + r) * D : k + (bs * la.Hkv + (r - la.H)) * D);
+            r < nq ? q + (bs * la.H + r) * D : k + (bs * la.Hkv + (r - nq)) * D);
         u0[u] = __ldg(src + c0);
         u1[u] = __ldg(src + c1);
       }
@@ -94,7 +115,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
     for (int u = 0; u < RB; ++u) {
       const int r = r0 + u;
       if (r >= nrows) break;  // uniform over the group
-      const bool is_q = r < la.H;
+      const bool is_q = r < nq;
       float x0[8], x1[8];
       unpack8(u0[u], x0);
       unpack8(u1[u], x1);
@@ -124,7 +145,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
           x1[e + 1] = b2 * c.z + a2 * c.w;
         }
       }
-      uint4* dst = reinterpret_cast<uint4*>(is_q ? qt + (bs * la.H + r) * D : kt + (bs * la.Hkv + (r - la.H)) * D);
+      uint4* dst = reinterpret_cast<uint4*>(is_q ? qt + (bs * la.H + r) * D : kt + (bs * la.Hkv + (r - nq)) * D);
       dst[c0] = pack8(x0);
       dst[c1] = pack8(x1);
     }
@@ -136,10 +157,63 @@ cudaError_t launch_qkprep(const bf16* q, const bf16* k, const int* positions, bf
   const long long tokens = static_cast<long long>(B) * S;
   const long long threads = tokens * (la.D / 16);
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  const ChunkPrep cp{nullptr, 0, 0};
   if (la.D == 256)
-    qkprep_kernel<16, 3><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status);
+    qkprep_kernel<16, 3, 0><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status, cp);
   else
-    qkprep_kernel<32, 3><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status);
+    qkprep_kernel<32, 3, 0><<<blocks, 256, 0, s>>>(q, k, positions, qt, kt, tokens, la, status, cp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qkprep_chunk(const bf16* q, const bf16* k_cache, const int* prefix, bf16* qt, bf16* kt,
+                                int B, int C, int max_len, const LayerArgs& la, uint32_t* status,
+                                cudaStream_t s) {
+  const ChunkPrep cp{prefix, C, max_len};
+  const long long tq = static_cast<long long>(B) * C, tk = static_cast<long long>(B) * max_len;
+  const unsigned bq = static_cast<unsigned>((tq * (la.D / 16) + 255) / 256);
+  const unsigned bk = static_cast<unsigned>((tk * (la.D / 16) + 255) / 256);
+  if (la.D == 256) {
+    qkprep_kernel<16, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
+    qkprep_kernel<16, 3, 1><<<bq, 256, 0, s>>>(q, nullptr, nullptr, qt, nullptr, tq, la, status, cp);
+  } else {
+    qkprep_kernel<32, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
+    qkprep_kernel<32, 3, 1><<<bq, 256, 0, s>>>(q, nullptr, nullptr, qt, nullptr, tq, la, status, cp);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Cache append: row (b, s, h) of the new rows to cache row (b, prefix[b] + s, h),
+// one 16-byte word per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                                        uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                                        const int* __restrict__ prefix, int C, int max_len,
+                                                        int row_words, long long words, uint32_t* status) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gid >= words) return;
+  const long long per_b = static_cast<long long>(C) * row_words;  // words of one sequence's new rows
+  const int b = static_cast<int>(gid / per_b);
+  const long long w = gid % per_b;
+  const int raw = __ldg(prefix + b);
+  const int pre = min(max(raw, 0), max_len - C);
+  if (w == 0 && pre != raw && status) flag_status(status, kStatusBounds);
+  const long long dst = (static_cast<long long>(b) * max_len + pre) * row_words + w;
+  k_cache[dst] = __ldg(k_new + gid);
+  if (v_new) v_cache[dst] = __ldg(v_new + gid);
+}
+
+cudaError_t launch_kv_append(const bf16* k_new, const bf16* v_new, bf16* k_cache, bf16* v_cache,
+                             const int* prefix, int B, int C, int max_len, int Hkv, int D, uint32_t* status,
+                             cudaStream_t s) {
+  const int row_words = Hkv * D / 8;  // one position's kv heads, in 16-byte words
+  const long long words = static_cast<long long>(B) * C * row_words;
+  if (words <= 0) return cudaSuccess;
+  const long long blocks = (words + 255) / 256;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new), reinterpret_cast<uint4*>(k_cache),
+      reinterpret_cast<uint4*>(v_cache), prefix, C, max_len, row_words, words, status);
   return cudaGetLastError();
 }
 

@@ -28,7 +28,7 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
            "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded", "gattn_kv_quantize",
-           "gattn_decode_int8")
+           "gattn_decode_int8", "gattn_prefill_chunk_workspace_size", "gattn_prefill_chunk", "gattn_kv_append")
 
 
 class GattnError(RuntimeError):
@@ -101,6 +101,13 @@ def lib() -> ctypes.CDLL:
         L.gattn_set_trace_buffer.argtypes = [vp, sz]
         L.gattn_decode_noalloc.restype = ctypes.c_int
         L.gattn_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp]
+        L.gattn_prefill_chunk_workspace_size.restype = sz
+        L.gattn_prefill_chunk_workspace_size.argtypes = [ctypes.POINTER(GattnCfg), i32, i32, i32]
+        L.gattn_prefill_chunk.restype = ctypes.c_int
+        L.gattn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.POINTER(GattnCfg), vp, sz,
+                                          vp]
+        L.gattn_kv_append.restype = ctypes.c_int
+        L.gattn_kv_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
         L.gattn_kv_quantize.restype = ctypes.c_int
         L.gattn_kv_quantize.argtypes = [vp, vp, vp, ctypes.c_int64, i32, vp]
         L.gattn_decode_int8.restype = ctypes.c_int
@@ -255,6 +262,35 @@ class AttentionLayer:
         return out
 
 
+    def prefill_chunk_workspace(self, batch: int, chunk_len: int, max_len: int, device="cuda") -> torch.Tensor:
+        n = lib().gattn_prefill_chunk_workspace_size(ctypes.byref(self.cfg), batch, chunk_len, max_len)
+        if n == 0:
+            raise GattnError(1, "gattn_prefill_chunk_workspace_size", "invalid cfg or sizes")
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+        _raise_if(lib().gattn_workspace_init(_ptr(ws), n, _stream()), "gattn_workspace_init")
+        return ws
+
+    def prefill_chunk(self, q, k_cache, v_cache=None, prefix_lens=None, k_new=None, v_new=None, out=None,
+                      workspace=None, stream=None):
+        """gattn_prefill_chunk: q [B,C,H,D] at positions prefix_lens[b] + i against caches
+        [B,Lmax,Hkv,D] (raw keys/values); k_new/v_new [B,C,Hkv,D] are appended first when given."""
+        _need(q, "q", torch.bfloat16, 4)
+        _need(k_cache, "k_cache", torch.bfloat16, 4)
+        if v_cache is not None:
+            _need(v_cache, "v_cache", torch.bfloat16, 4)
+        for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+            if t is not None:
+                _need(t, n, torch.bfloat16, 4)
+        _need(prefix_lens, "prefix_lens", torch.int32, 1)
+        B, C = q.shape[0], q.shape[1]
+        Lmax = k_cache.shape[1]
+        out = torch.empty_like(q) if out is None else out
+        ws = self.prefill_chunk_workspace(B, C, Lmax, q.device) if workspace is None else workspace
+        _raise_if(lib().gattn_prefill_chunk(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                            _ptr(prefix_lens), _ptr(out), B, C, Lmax, ctypes.byref(self.cfg),
+                                            _ptr(ws), ws.numel(), _stream(stream)), "gattn_prefill_chunk")
+        return out
+
     def decode_int8(self, q, k_codes, k_scales, v_codes=None, v_scales=None, seq_lens=None, out=None,
                     workspace=None, stream=None):
         """gattn_decode_int8: q [B,H,D] bf16; codes [B,Lmax,Hkv,D] int8 and scales [B,Lmax,Hkv] fp32
@@ -277,6 +313,19 @@ class AttentionLayer:
                                           _ptr(seq_lens), _ptr(out), B, Lmax, ctypes.byref(self.cfg), _ptr(ws),
                                           ws.numel(), _stream(stream)), "gattn_decode_int8")
         return out
+
+
+def kv_append(k_new, v_new, k_cache, v_cache, cache_lens, status=None, stream=None):
+    """gattn_kv_append: rows [B,n,Hkv,D] into caches [B,Lmax,Hkv,D] at rows [cache_lens[b], +n)."""
+    _need(k_new, "k_new", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    if v_new is not None:
+        _need(v_new, "v_new", torch.bfloat16, 4)
+        _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(cache_lens, "cache_lens", torch.int32, 1)
+    B, n, Hkv, D = k_new.shape
+    _raise_if(lib().gattn_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), B, n,
+                                    k_cache.shape[1], Hkv, D, _ptr(status), _stream(stream)), "gattn_kv_append")
 
 
 def kv_quantize(x: torch.Tensor, codes=None, scales=None, stream=None):

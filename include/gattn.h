@@ -139,11 +139,52 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
  * rows of padding tokens are zero.  Positions of padding tokens must still be
  * in [0, rope_max_pos) (they are rotated, then ignored).  Every other argument,
  * the workspace size and the errors are those of gattn_prefill; with every
- * range [0, seq_len) the result is bit-identical to gattn_prefill's. */
+ * range [0, seq_len) the result is bit-identical to gattn_prefill's.  Padding
+ * rows of k and v get weight exactly 0 but are read: they must be finite. */
 int gattn_prefill_padded(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
                          const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,
                          int32_t batch, int32_t seq_len, const gattn_cfg* cfg, void* workspace,
                          size_t ws_bytes, gattn_stream stream);
+
+/* ---- a chunk of a prompt against a cached prefix ------------------------------
+ * The generate loop of KerasFormers "Gemma 4" (Gemma4Generate.generate) runs a
+ * prompt, then tokens one by one, over a KV cache; a chunk is the step between:
+ * C new tokens of sequence b at positions P_b .. P_b + C - 1 (P_b =
+ * prefix_lens[b], the tokens already cached), each attending to the cache rows
+ * [0, P_b + i] (within the window).  Caches hold RAW keys/values as in
+ * gattn_decode, cached key j at position j.
+ *   q               [batch][C][H][D] bf16, the chunk's queries (before QK-norm/RoPE)
+ *   k_new, v_new    [batch][C][Hkv][D] bf16, the chunk's raw keys/values: copied into
+ *                   cache rows [P_b, P_b + C) first (the cache append); both NULL
+ *                   when those rows are already in the cache (v_new NULL with k_eq_v)
+ *   k_cache, v_cache_or_null [batch][max_len][Hkv][D] bf16 (device, written by the append)
+ *   prefix_lens     [batch] int32 (device): P_b in [0, max_len - C]; outside it is
+ *                   clamped and flags GATTN_ERR_DEVICE_BOUNDS
+ *   out             [batch][C][H][D] bf16
+ * With C = the whole prompt and P_b = 0 it is gattn_prefill over the cache rows.
+ * workspace: at least gattn_prefill_chunk_workspace_size(cfg, batch, C, max_len)
+ * bytes (the transformed cache keys and chunk queries when QK-norm or RoPE is on).
+ * Errors as gattn_prefill; the positions used by RoPE must be below rope_max_pos.
+ * Cache rows past P_b + C are never weighted, but the last key tile of a chunk
+ * reads up to 127 of them (weight exactly 0): they must hold finite values
+ * (a zero-initialised cache does); rows beyond the tile are not read. */
+size_t gattn_prefill_chunk_workspace_size(const gattn_cfg* cfg, int32_t batch, int32_t chunk_len, int32_t max_len);
+int gattn_prefill_chunk(const gattn_bf16* q, const gattn_bf16* k_new_or_null, const gattn_bf16* v_new_or_null,
+                        gattn_bf16* k_cache, gattn_bf16* v_cache_or_null, const int32_t* prefix_lens,
+                        gattn_bf16* out, int32_t batch, int32_t chunk_len, int32_t max_len, const gattn_cfg* cfg,
+                        void* workspace, size_t ws_bytes, gattn_stream stream);
+
+/* gattn_kv_append: the cache append alone (e.g. before gattn_decode of a new token):
+ * rows [batch][n_new][Hkv][D] bf16 of k_new (and v_new) into cache rows
+ * [cache_lens[b], cache_lens[b] + n_new) of [batch][max_len][Hkv][D] caches.
+ * cache_lens (device int32) are the rows held before the append; a value outside
+ * [0, max_len - n_new] is clamped and, when status_or_null is a gattn workspace,
+ * flags GATTN_ERR_DEVICE_BOUNDS there (read with gattn_check).  v_new and v_cache
+ * are both NULL or both given; rows 16-byte aligned; head_dim a multiple of 8. */
+int gattn_kv_append(const gattn_bf16* k_new, const gattn_bf16* v_new_or_null, gattn_bf16* k_cache,
+                    gattn_bf16* v_cache_or_null, const int32_t* cache_lens, int32_t batch, int32_t n_new,
+                    int32_t max_len, int32_t num_kv_heads, int32_t head_dim, void* status_or_null,
+                    gattn_stream stream);
 
 /* ---- decode ----------------------------------------------------------------
  * One decode step: query b (at position seq_lens[b]-1) against cache rows

@@ -237,7 +237,7 @@ def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, bat
     return out
 
 
-def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k=None):
+def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k=None, rows=None):
     """A chunk of C new tokens against a cached prefix (float64): the prompt in pieces.
 
     KerasFormers "Gemma 4", Gemma4Generate.generate runs the model over a prompt
@@ -248,23 +248,24 @@ def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k
     [0, P_b + i] (within the window), cached key j at position j (raw keys and
     values, as attention_decode takes them).
     q [B,C,H,D]; k_cache / v_cache [B,Lmax,Hkv,D] (v_cache None when k_eq_v).
-    Returns [B,C,H,D].
+    ``rows`` optionally restricts the output to those chunk rows.  Returns [B,R,H,D].
     """
     f = _layer_fields(cfg)
     q = _f64(q)
     B, C, H, D = q.shape
     G = H // f["Hkv"]
     prefix_lens = np.asarray(_f64(prefix_lens)).astype(np.int64)
-    out = np.zeros((B, C, H, D))
+    rows = np.arange(C) if rows is None else np.asarray(rows)
+    out = np.zeros((B, len(rows), H, D))
     for b in range(B):
         P = int(prefix_lens[b])
         n = P + C                                   # cache rows the chunk can see
         kc = _f64(k_cache[b])[:n]
         vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:n]
         k_idx = np.arange(n)                        # cached key j: token j, position j
-        q_idx = P + np.arange(C)                    # chunk token i: token P + i
+        q_idx = P + rows                            # chunk token i: token P + i
         kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), k_idx[:, None], f["rot"], f["theta"], f["F"])
-        qt = rope(rms_norm(q[b], w_q, f["mode"], f["eps"]), q_idx[:, None], f["rot"], f["theta"], f["F"])
+        qt = rope(rms_norm(q[b, rows], w_q, f["mode"], f["eps"]), q_idx[:, None], f["rot"], f["theta"], f["F"])
         for h in range(H):
             kv = h // G
             out[b, :, h] = _attend(qt[:, h], kt[:, kv], vc[:, kv], q_idx, k_idx, f["scale"], f["cap"], f["W"])

@@ -137,6 +137,43 @@ def test_decode_int8_rejects_bad_args():
     assert decode_int8(c, B=0) == 0
 
 
+def prefill_chunk(c, q=ALIGNED, kn=ALIGNED, vn=ALIGNED, kc=ALIGNED, vc=ALIGNED, pre=ALIGNED, out=ALIGNED, B=1, C=16,
+                  Lmax=64, ws=ALIGNED, ws_bytes=1 << 30):
+    return G.lib().gattn_prefill_chunk(q, kn, vn, kc, vc, pre, out, B, C, Lmax, ctypes.byref(c), ws, ws_bytes, None)
+
+
+def test_prefill_chunk_rejects_bad_args():
+    c = cfg()
+    assert prefill_chunk(c, C=65) == INVALID                    # chunk longer than the cache
+    assert prefill_chunk(c, pre=None) == INVALID
+    assert prefill_chunk(c, pre=ALIGNED + 2) == INVALID
+    assert prefill_chunk(c, kc=ALIGNED + 8) == INVALID
+    assert prefill_chunk(c, vn=None) == INVALID                  # k_new without v_new
+    assert prefill_chunk(c, vc=None) == INVALID
+    assert prefill_chunk(cfg(head_dim=128)) == UNSUPPORTED
+    assert prefill_chunk(c, ws_bytes=16) == WORKSPACE
+    assert prefill_chunk(c, B=0) == 0 and prefill_chunk(c, C=0) == 0
+    assert prefill_chunk(c, kn=None, vn=None, B=0) == 0
+    ck = cfg(k_eq_v=1)
+    assert prefill_chunk(ck, vc=ALIGNED + 4096) == INVALID      # tied: v_cache NULL or k_cache
+    n_small = G.lib().gattn_prefill_chunk_workspace_size(ctypes.byref(c), 2, 16, 64)
+    cr = cfg(rotary_fraction=1.0, rope_table=ALIGNED, rope_max_pos=64)
+    n_rope = G.lib().gattn_prefill_chunk_workspace_size(ctypes.byref(cr), 2, 16, 64)
+    assert n_small >= 4 and n_rope >= 2 * 64 * 1 * 256 * 2 + 2 * 16 * 8 * 256 * 2
+    assert G.lib().gattn_prefill_chunk_workspace_size(ctypes.byref(c), 2, 65, 64) == 0
+
+
+def test_kv_append_rejects_bad_args():
+    L = G.lib()
+    f = L.gattn_kv_append
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 1, 17, 16, 2, 256, None, None) == INVALID  # n_new > max_len
+    assert f(ALIGNED, None, ALIGNED, ALIGNED, ALIGNED, 1, 4, 16, 2, 256, None, None) == INVALID   # v_new xor v_cache
+    assert f(ALIGNED + 8, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 1, 4, 16, 2, 256, None, None) == INVALID
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED + 2, 1, 4, 16, 2, 256, None, None) == INVALID
+    assert f(ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 1, 4, 16, 2, 100, None, None) == INVALID  # head_dim % 8
+    assert f(None, None, None, None, None, 0, 4, 16, 2, 256, None, None) == 0                    # empty
+
+
 def test_empty_problem_is_a_no_op():
     assert prefill(cfg(), B=0) == 0
     assert prefill(cfg(), S=0) == 0

@@ -83,8 +83,8 @@ MUTATIONS = {
         [T8.test_round_trip_within_half_step_and_extremes,
          T8.test_int8_decode_equals_float_decode_on_representable_cache]),
     "chunk_queries_at_local_positions": (
-        "q_idx = P + np.arange(C)                    # chunk token i: token P + i",
-        "q_idx = np.arange(C)",
+        "q_idx = P + rows                            # chunk token i: token P + i",
+        "q_idx = rows",
         [TC.test_chunk_equals_rows_of_whole_prompt, TC.test_chunk_onehot_counts]),
     "chunk_sees_only_prefix": (
         "n = P + C                                   # cache rows the chunk can see", "n = max(P, 1)",

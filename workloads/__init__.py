@@ -76,6 +76,20 @@ class PrefillWorkload:
 
 
 @dataclasses.dataclass(frozen=True)
+class ChunkWorkload:
+    """The last ``chunk`` tokens of a ``prefix + chunk`` prompt, the first ``prefix``
+    already in the cache (KerasFormers "Gemma 4", Gemma4Generate.generate, in pieces)."""
+    name: str
+    layer: Layer
+    batch: int
+    prefix: int
+    chunk: int
+    seed: int
+    gain_mean: float = 0.0
+    gain_std: float = 0.1
+
+
+@dataclasses.dataclass(frozen=True)
 class DecodeWorkload:
     name: str
     layer: Layer
@@ -152,6 +166,11 @@ GEMMA3_GLOBAL_LEFTPAD = PrefillWorkload(
 GEMMA4_DECODE_LOCAL_INT8 = dataclasses.replace(GEMMA4_DECODE_LOCAL, name="gemma4_12b_decode_local_int8_b64",
                                                kv_int8=True)
 
+# the last 1024-token chunk of eight 8192-token prompts through the Gemma 3 global layer
+GEMMA3_GLOBAL_CHUNK = ChunkWorkload(
+    "gemma3_1b_global_b8_chunk1024_prefix7168",
+    Layer(window=0, rope_theta=1e6, **_G3), batch=8, prefix=7168, chunk=1024, seed=6)
+
 PREFILL: Dict[str, PrefillWorkload] = {w.name: w for w in (
     GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL, GEMMA3_GLOBAL_LEFTPAD)}
 DECODE: Dict[str, DecodeWorkload] = {w.name: w for w in (
@@ -202,6 +221,24 @@ def prefill_inputs(wl: PrefillWorkload, batch: Optional[int] = None,
         positions = torch.clamp(t - lo.unsqueeze(1), min=0).to(torch.int32).contiguous()
     return dict(q=q, k=k, v=v, positions=positions, w_q=w_q, w_k=w_k, layer=layer,
                 seq_range=seq_range)
+
+
+def chunk_inputs(wl: ChunkWorkload) -> dict:
+    """The whole prompt drawn as a prefill of prefix + chunk tokens (same draw order),
+    split into the cache (rows [0, prefix), zeros past them) and the chunk's q, k, v."""
+    n = wl.prefix + wl.chunk
+    d = prefill_inputs(PrefillWorkload(wl.name, wl.layer, wl.batch, n, wl.seed, wl.gain_mean, wl.gain_std))
+    P, C = wl.prefix, wl.chunk
+    k_cache = torch.zeros_like(d["k"])
+    k_cache[:, :P] = d["k"][:, :P]
+    v_cache = None
+    if d["v"] is not None:
+        v_cache = torch.zeros_like(d["v"])
+        v_cache[:, :P] = d["v"][:, :P]
+    return dict(q=d["q"][:, P:].contiguous(), k_new=d["k"][:, P:].contiguous(),
+                v_new=None if d["v"] is None else d["v"][:, P:].contiguous(), k_cache=k_cache, v_cache=v_cache,
+                prefix_lens=torch.full((wl.batch,), P, dtype=torch.int32), w_q=d["w_q"], w_k=d["w_k"],
+                layer=wl.layer, max_len=n)
 
 
 def decode_inputs(wl: DecodeWorkload, batch: Optional[int] = None,
