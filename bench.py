@@ -283,6 +283,18 @@ def make_chunk(wl, dev):
                             "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 
+def dominant_decode_src(L: W.Layer) -> str:
+    """Source of the split kernel a decode layer runs (the step's dominant kernel): the
+    tensor-core one for K=V with 8 or 16 query heads per kv head, the CUDA-core one for
+    1, 2 or 4, else the fallback in the prologue/combine file."""
+    G = L.num_heads // L.num_kv_heads
+    if L.k_eq_v and G in (8, 16):
+        return "gemma_family_decoder_b200/csrc/decode_tc.cu"
+    if G in (1, 2, 4):
+        return "gemma_family_decoder_b200/csrc/decode_simt.cu"
+    return "gemma_family_decoder_b200/csrc/prep_decode.cu"
+
+
 def make_decode(wl, dev):
     from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
     dq = W.decode_inputs(wl)
@@ -322,10 +334,7 @@ def make_decode(wl, dev):
     return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
                 work=decode_bytes(L, lens.numpy(), wl.kv_int8), unit="GB/s", scale=1e9,
                 metric="decode KV GB/s (algorithmic bytes)", bound="hbm", launches=2,
-                kernel_src=("gemma_family_decoder_b200/csrc/prep_decode.cu",
-                            "gemma_family_decoder_b200/csrc/decode_tc.cu",
-                            "gemma_family_decoder_b200/csrc/decode_simt.cu",
-                            "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
+                kernel_src=(dominant_decode_src(L), "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 
 def run_ours(args, world, rank, local):
