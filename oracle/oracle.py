@@ -202,7 +202,7 @@ def attention_prefill(q, k, v, positions, cfg, w_q=None, w_k=None, rows=None, se
 # --- the layer: one decode step ----------------------------------------------
 
 def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, batches=None,
-                     first_rows=None):
+                     first_rows=None, keys_transformed=False):
     """One decode step (float64): query b at position L_b - 1 over cache rows [0, L_b).
 
     q [B,H,D]; k_cache / v_cache [B,Lmax,Hkv,D] raw (un-normed, un-rotated)
@@ -210,7 +210,9 @@ def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, bat
     sits at position j.  ``batches`` restricts the output to those batch rows.
     ``first_rows[b]`` (default 0) says the cache given for batch row b starts
     at row first_rows[b]; the rows left out must all be masked, which is
-    asserted.  Returns [len(batches),H,D].
+    asserted.  ``keys_transformed``: the cache holds the keys after QK-norm and RoPE
+    (k~ of step 2, cached key j rotated at position j), used as they are; only
+    for layers whose values are not the keys.  Returns [len(batches),H,D].
     """
     f = _layer_fields(cfg)
     q = _f64(q)
@@ -226,8 +228,12 @@ def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, bat
         kc = _f64(k_cache[b])[:L - r0]
         vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:L - r0]
         pos_k = np.arange(r0, L)
-        kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],
-                  f["rot"], f["theta"], f["F"])
+        if keys_transformed:
+            assert not f["k_eq_v"], "tied values need the raw keys"
+            kt = kc
+        else:
+            kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],
+                      f["rot"], f["theta"], f["F"])
         qt = rope(rms_norm(q[b], w_q, f["mode"], f["eps"]), np.array([L - 1]),
                   f["rot"], f["theta"], f["F"])                       # [H,D]
         for h in range(H):
@@ -237,7 +243,8 @@ def attention_decode(q, k_cache, v_cache, seq_lens, cfg, w_q=None, w_k=None, bat
     return out
 
 
-def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k=None, rows=None):
+def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k=None, rows=None,
+                            keys_transformed=False):
     """A chunk of C new tokens against a cached prefix (float64): the prompt in pieces.
 
     KerasFormers "Gemma 4", Gemma4Generate.generate runs the model over a prompt
@@ -248,7 +255,8 @@ def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k
     [0, P_b + i] (within the window), cached key j at position j (raw keys and
     values, as attention_decode takes them).
     q [B,C,H,D]; k_cache / v_cache [B,Lmax,Hkv,D] (v_cache None when k_eq_v).
-    ``rows`` optionally restricts the output to those chunk rows.  Returns [B,R,H,D].
+    ``rows`` optionally restricts the output to those chunk rows;
+    ``keys_transformed`` as in attention_decode.  Returns [B,R,H,D].
     """
     f = _layer_fields(cfg)
     q = _f64(q)
@@ -264,12 +272,24 @@ def attention_prefill_chunk(q, k_cache, v_cache, prefix_lens, cfg, w_q=None, w_k
         vc = kc if f["k_eq_v"] else _f64(v_cache[b])[:n]
         k_idx = np.arange(n)                        # cached key j: token j, position j
         q_idx = P + rows                            # chunk token i: token P + i
-        kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), k_idx[:, None], f["rot"], f["theta"], f["F"])
+        if keys_transformed:
+            assert not f["k_eq_v"], "tied values need the raw keys"
+            kt = kc
+        else:
+            kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), k_idx[:, None], f["rot"], f["theta"], f["F"])
         qt = rope(rms_norm(q[b, rows], w_q, f["mode"], f["eps"]), q_idx[:, None], f["rot"], f["theta"], f["F"])
         for h in range(H):
             kv = h // G
             out[b, :, h] = _attend(qt[:, h], kt[:, kv], vc[:, kv], q_idx, k_idx, f["scale"], f["cap"], f["W"])
     return out
+
+
+def transform_keys(k_rows, positions, cfg, w_k=None):
+    """The keys a transformed cache holds: RoPE(QK-norm(k)) of rows k_rows [N,Hkv,D] at
+    ``positions`` [N] (steps 1-2), float64."""
+    f = _layer_fields(cfg)
+    return rope(rms_norm(_f64(k_rows), w_k, f["mode"], f["eps"]), np.asarray(positions)[:, None],
+                f["rot"], f["theta"], f["F"])
 
 
 # --- split-KV merge (decode's two-stage form) ---------------------------------
@@ -323,7 +343,7 @@ def kv_dequantize(codes, scales):
 
 
 def attention_decode_int8(q, k_codes, k_scales, v_codes, v_scales, seq_lens, cfg, w_q=None, w_k=None,
-                          batches=None, first_rows=None):
+                          batches=None, first_rows=None, keys_transformed=False):
     """One decode step over an int8 cache: attention_decode on the dequantised rows.
 
     k_codes / v_codes [B,Lmax,Hkv,D] int8 (or per-batch lists, as attention_decode
@@ -338,4 +358,4 @@ def attention_decode_int8(q, k_codes, k_scales, v_codes, v_scales, seq_lens, cfg
     kd = deq(k_codes, k_scales)
     vd = None if f["k_eq_v"] else deq(v_codes, v_scales)
     return attention_decode(q, kd, vd, seq_lens, cfg, w_q=w_q, w_k=w_k, batches=batches,
-                            first_rows=first_rows)
+                            first_rows=first_rows, keys_transformed=keys_transformed)

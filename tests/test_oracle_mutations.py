@@ -15,6 +15,7 @@ import oracle.oracle as src_mod
 import test_oracle as T
 import test_oracle_int8 as T8
 import test_oracle_chunk as TC
+import test_oracle_transformed as TT
 
 MUTATIONS = {
     # name: (original text, replacement, pins that must fail)
@@ -89,6 +90,16 @@ MUTATIONS = {
     "chunk_sees_only_prefix": (
         "n = P + C                                   # cache rows the chunk can see", "n = max(P, 1)",
         [TC.test_chunk_equals_rows_of_whole_prompt]),
+    "transformed_keys_normed_again": (
+        """            assert not f["k_eq_v"], "tied values need the raw keys"
+            kt = kc
+        else:
+            kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],""",
+        """            assert not f["k_eq_v"], "tied values need the raw keys"
+            kt = rms_norm(kc, w_k, f["mode"], f["eps"])
+        else:
+            kt = rope(rms_norm(kc, w_k, f["mode"], f["eps"]), pos_k[:, None],""",
+        [TT.test_decode_over_transformed_keys_equals_raw]),
     "int8_values_from_key_codes": (
         "else deq(v_codes, v_scales)", "else deq(k_codes, v_scales)",
         [T8.test_int8_decode_equals_float_decode_on_representable_cache]),
