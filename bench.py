@@ -46,8 +46,9 @@ PREFILL_WL = {
     "gemma3_1b_global_b8_s4096_leftpad": W.GEMMA3_GLOBAL_LEFTPAD,
 }
 DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
-                                 W.GEMMA4_DECODE_GLOBAL_NORM, W.GEMMA4_DECODE_LOCAL_INT8)}
-CHUNK_WL = {W.GEMMA3_GLOBAL_CHUNK.name: W.GEMMA3_GLOBAL_CHUNK}
+                                 W.GEMMA4_DECODE_GLOBAL_NORM, W.GEMMA4_DECODE_LOCAL_INT8,
+                                 W.GEMMA4_DECODE_LOCAL_TK, W.GEMMA4_DECODE_LOCAL_INT8_TK)}
+CHUNK_WL = {w.name: w for w in (W.GEMMA3_GLOBAL_CHUNK, W.GEMMA3_GLOBAL_CHUNK_TK)}
 HEADLINE = "gemma1_2b_mqa_b4_s2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -260,11 +261,19 @@ def make_prefill(wl, dev):
 def make_chunk(wl, dev):
     from gemma_family_decoder_b200 import AttentionLayer, LayerSpec
     d = W.chunk_inputs(wl)
-    layer = AttentionLayer(LayerSpec.of(wl.layer), d["max_len"], d["w_q"], d["w_k"], device=dev)
+    spec = dataclasses.replace(LayerSpec.of(wl.layer), keys_transformed=wl.keys_transformed)
+    layer = AttentionLayer(spec, d["max_len"], d["w_q"], d["w_k"], device=dev)
     host = {k: d[k].pin_memory() for k in ("q", "k_new", "v_new", "prefix_lens") if d[k] is not None}
     devt = {k: t.to(dev) for k, t in host.items()}
     k_cache = d["k_cache"].to(dev)
     v_cache = None if d["v_cache"] is None else d["v_cache"].to(dev)
+    if wl.keys_transformed:
+        # the cached prefix as the library's append writes it: keys normed and rotated
+        full_k = torch.zeros_like(k_cache)
+        full_v = torch.zeros_like(v_cache)
+        layer.kv_append(k_cache[:, :wl.prefix].contiguous(), v_cache[:, :wl.prefix].contiguous(), full_k, full_v,
+                        torch.zeros(wl.batch, dtype=torch.int32, device=dev))
+        k_cache, v_cache = full_k, full_v
     out = torch.empty_like(devt["q"])
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     ws = layer.prefill_chunk_workspace(wl.batch, wl.chunk, d["max_len"], dev)
@@ -310,7 +319,19 @@ def make_decode(wl, dev):
         k[b, lo:n] = rows["k"].to(dev)
         if v is not None:
             v[b, lo:n] = rows["v"].to(dev)
-    layer = AttentionLayer(LayerSpec.of(L), wl.max_len, dq["w_q"], dq["w_k"], device=dev)
+    spec = dataclasses.replace(LayerSpec.of(L), keys_transformed=wl.keys_transformed)
+    layer = AttentionLayer(spec, wl.max_len, dq["w_q"], dq["w_k"], device=dev)
+    if wl.keys_transformed:
+        # the same rows as the library's append writes them: keys normed and rotated
+        kt = torch.zeros_like(k)
+        v_scratch = torch.empty_like(v[:1])  # the append's value copy, not needed here
+        for b in range(wl.batch):
+            n = int(lens[b])
+            lo = 0 if L.window == 0 else max(0, n - L.window)
+            layer.kv_append(k[b:b + 1, lo:n].contiguous(), v[b:b + 1, lo:n].contiguous(), kt[b:b + 1], v_scratch,
+                            torch.tensor([lo], dtype=torch.int32, device=dev))
+        del v_scratch
+        k = kt
     host = {"q": dq["q"].pin_memory(), "seq_lens": lens.pin_memory()}
     devt = {"q": host["q"].to(dev), "seq_lens": host["seq_lens"].to(dev), "k": k, "v": v}
     out = torch.empty_like(devt["q"])
@@ -482,15 +503,20 @@ def _oracle_prefill_rows(wl, d, rows):
                         w_k=d["w_k"], rows=rows, seq_range=d.get("seq_range"))
 
 
-def _oracle_cache(wl, ks, vs):
-    """The oracle's cache rows per batch row (None where left out): bf16 as drawn, or, for an
-    int8 workload, the oracle's own codes and scales of them."""
+def _oracle_cache(wl, ks, vs, firsts):
+    """The oracle's cache rows per batch row (None where left out): bf16 as drawn (keys
+    transformed by the oracle for a transformed-key workload), or, for an int8 workload,
+    the oracle's own codes and scales of them."""
     import oracle as O
+    if wl.keys_transformed:
+        ks = [None if r is None else O.transform_keys(r, np.arange(firsts[b], firsts[b] + len(r)), wl.layer)
+              for b, r in enumerate(ks)]
     if not wl.kv_int8:
         return dict(k=ks, v=vs)
 
     def q8(rows):
-        cs = [None if r is None else O.kv_quantize(r.float().numpy()) for r in rows]
+        cs = [None if r is None else O.kv_quantize(r.float().numpy() if torch.is_tensor(r) else np.asarray(r))
+              for r in rows]
         return [None if c is None else c[0] for c in cs], [None if c is None else c[1] for c in cs]
 
     kc, ksc = q8(ks)
@@ -503,9 +529,11 @@ def _oracle_decode(wl, dq, cache, batches, firsts):
     L = wl.layer
     if wl.kv_int8:
         return O.attention_decode_int8(dq["q"], cache["kc"], cache["ks"], cache["vc"], cache["vs"], dq["seq_lens"],
-                                       L, w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts)
+                                       L, w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts,
+                                       keys_transformed=wl.keys_transformed)
     return O.attention_decode(dq["q"], cache["k"], None if L.k_eq_v else cache["v"], dq["seq_lens"], L,
-                              w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts)
+                              w_q=dq["w_q"], w_k=dq["w_k"], batches=batches, first_rows=firsts,
+                              keys_transformed=wl.keys_transformed)
 
 
 def _oracle_chunk(wl, d, rows):
@@ -574,7 +602,7 @@ def cpu_baseline(name, budget_s=15.0):
         ks.append(rows["k"])
         vs.append(rows["v"])
         firsts.append(lo)
-    cache = _oracle_cache(wl, ks, vs)
+    cache = _oracle_cache(wl, ks, vs, firsts)
     t0 = time.perf_counter()
     for b in range(wl.batch):
         _oracle_decode(wl, dq, cache, [b], firsts)
@@ -650,7 +678,7 @@ def run_reference(args, world, rank):
             ks = [rows["k"] if j == b else None for j in range(wl.batch)]
             vs = [rows["v"] if j == b else None for j in range(wl.batch)]
             fr = [lo if j == b else 0 for j in range(wl.batch)]
-            cache = _oracle_cache(wl, ks, vs)
+            cache = _oracle_cache(wl, ks, vs, fr)
             t0 = time.perf_counter()
             _oracle_decode(wl, dq, cache, [b], fr)
             el = time.perf_counter() - t0

@@ -328,8 +328,11 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
   const uint64_t tmo = P.timeout_ns;
   const size_t row_elems = static_cast<size_t>(Hkv) * D;  // one cache position
   const int half = la.rot >> 1;
+  // a cache of transformed keys: no key norm and no key rotation
+  const bool knorm = la.qk_norm && !la.kt_cache;
+  const int khalf = la.kt_cache ? 0 : half;
   // the (cos, sin) rows of a tile's positions travel with the tile when they fit
-  const bool tab_staged = half > 0 && TP * half * static_cast<int>(sizeof(float2)) <= kTabBytes;
+  const bool tab_staged = khalf > 0 && TP * half * static_cast<int>(sizeof(float2)) <= kTabBytes;
 
   // ------------------------------------------------------------ tile copies
   // Stage st of tile u is refilled with tile u + NST by the last warp to finish
@@ -510,7 +513,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
             else zero_lane2<NC>(k2[r]);
           }
         }
-        if (la.qk_norm) {
+        if (knorm) {
 #pragma unroll
           for (int r = 0; r < RB; ++r) {
             float2 a2 = __fmul2_rn(k2[r][0][0], k2[r][0][0]);
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
             }
           }
         }
-        if (half > 0) {
+        if (khalf > 0) {
           // the position's table row: staged with the tile (shared-memory
           // loads), else from global memory (positions past the table flagged
           // and clamped); two separate loops so that each load has one space
@@ -576,7 +579,7 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
           }
       }
       float x = transpose_sum<NV>(part, lane);
-      if (la.qk_norm) {
+      if (knorm) {
         // 1/rms of each row: sums of squares through the same butterfly, then
         // each row's factor from the warp scratch
         float s2 = transpose_sum<RPW>(ssr, lane);

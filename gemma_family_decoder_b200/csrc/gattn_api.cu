@@ -71,6 +71,10 @@ int resolve(const gattn_cfg* cfg, gattn::LayerArgs* la, bool need_ptrs) {
   if (!(cfg->scalar > 0.f) || std::isinf(cfg->scalar))
     return fail(GATTN_ERR_INVALID_ARG, "scalar must be finite and > 0");
   if (cfg->k_eq_v != 0 && cfg->k_eq_v != 1) return fail(GATTN_ERR_INVALID_ARG, "k_eq_v must be 0 or 1");
+  if (cfg->keys_transformed != 0 && cfg->keys_transformed != 1)
+    return fail(GATTN_ERR_INVALID_ARG, "keys_transformed must be 0 or 1");
+  if (cfg->keys_transformed && cfg->k_eq_v)
+    return fail(GATTN_ERR_INVALID_ARG, "keys_transformed with k_eq_v: tied values need the raw keys");
   if (cfg->qk_norm < 0 || cfg->qk_norm > 2) return fail(GATTN_ERR_INVALID_ARG, "qk_norm must be 0, 1 or 2");
   if (cfg->qk_norm != 0) {
     if (!(cfg->norm_eps >= 0.f)) return fail(GATTN_ERR_INVALID_ARG, "norm_eps must be >= 0");
@@ -97,6 +101,7 @@ int resolve(const gattn_cfg* cfg, gattn::LayerArgs* la, bool need_ptrs) {
   la->q_norm_w = cfg->q_norm_w;
   la->k_norm_w = cfg->k_norm_w;
   la->k_eq_v = cfg->k_eq_v;
+  la->kt_cache = cfg->keys_transformed;
   return GATTN_OK;
 }
 
@@ -359,6 +364,40 @@ int gattn_kv_append(const gattn_bf16* k_new, const gattn_bf16* v_new_or_null, ga
   return GATTN_OK;
 }
 
+int gattn_kv_append_layer(const gattn_cfg* cfg, const gattn_bf16* k_new, const gattn_bf16* v_new_or_null,
+                          gattn_bf16* k_cache, gattn_bf16* v_cache_or_null, const int32_t* cache_lens,
+                          int32_t batch, int32_t n_new, int32_t max_len, void* status_or_null,
+                          gattn_stream stream) {
+  g_last_error[0] = 0;
+  gattn::LayerArgs la;
+  int st = resolve(cfg, &la, true);
+  if (st != GATTN_OK) return st;
+  if (!la.kt_cache || !prefill_needs_kprep(la))
+    return gattn_kv_append(k_new, v_new_or_null, k_cache, v_cache_or_null, cache_lens, batch, n_new, max_len, la.Hkv,
+                           la.D, status_or_null, stream);
+  if (batch < 0 || n_new < 0 || max_len < n_new)
+    return fail(GATTN_ERR_INVALID_ARG, "need batch, n_new >= 0 and max_len >= n_new");
+  if (batch == 0 || n_new == 0) return GATTN_OK;
+  if (!k_new || !k_cache || !cache_lens || !v_new_or_null || !v_cache_or_null)
+    return fail(GATTN_ERR_INVALID_ARG, "k_new, v_new, k_cache, v_cache and cache_lens must not be NULL");
+  if (!aligned16(k_new) || !aligned16(k_cache) || !aligned16(v_new_or_null) || !aligned16(v_cache_or_null))
+    return fail(GATTN_ERR_INVALID_ARG, "rows must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(cache_lens) & 3u) return fail(GATTN_ERR_INVALID_ARG, "cache_lens must be 4-byte aligned");
+  if (status_or_null && !aligned16(status_or_null)) return fail(GATTN_ERR_INVALID_ARG, "status must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(status_or_null);
+  cudaError_t e = gattn::launch_kv_append(nullptr, reinterpret_cast<const __nv_bfloat16*>(v_new_or_null),
+                                          reinterpret_cast<__nv_bfloat16*>(k_cache),
+                                          reinterpret_cast<__nv_bfloat16*>(v_cache_or_null), cache_lens, batch, n_new,
+                                          max_len, la.Hkv, la.D, status, s);
+  if (e == cudaSuccess)
+    e = gattn::launch_key_append_transformed(reinterpret_cast<const __nv_bfloat16*>(k_new),
+                                             reinterpret_cast<__nv_bfloat16*>(k_cache), cache_lens, batch, n_new,
+                                             max_len, la, status, s);
+  if (e != cudaSuccess) return fail_cuda(e, "kv append launch");
+  return GATTN_OK;
+}
+
 int gattn_prefill_chunk(const gattn_bf16* q, const gattn_bf16* k_new_or_null, const gattn_bf16* v_new_or_null,
                         gattn_bf16* k_cache, gattn_bf16* v_cache_or_null, const int32_t* prefix_lens,
                         gattn_bf16* out, int32_t batch, int32_t chunk_len, int32_t max_len, const gattn_cfg* cfg,
@@ -397,11 +436,17 @@ int gattn_prefill_chunk(const gattn_bf16* q, const gattn_bf16* k_new_or_null, co
   uint32_t* status = static_cast<uint32_t*>(workspace);
   __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(k_cache);
   __nv_bfloat16* vc = la.k_eq_v ? kc : reinterpret_cast<__nv_bfloat16*>(v_cache_or_null);
+  // a transformed cache receives the chunk's keys normed and rotated, and its
+  // keys are read as they are
+  const bool kt_cache = la.kt_cache && prefill_needs_kprep(la);
   if (k_new_or_null) {
     cudaError_t e = gattn::launch_kv_append(
-        reinterpret_cast<const __nv_bfloat16*>(k_new_or_null),
+        kt_cache ? nullptr : reinterpret_cast<const __nv_bfloat16*>(k_new_or_null),
         la.k_eq_v ? nullptr : reinterpret_cast<const __nv_bfloat16*>(v_new_or_null), kc, la.k_eq_v ? nullptr : vc,
         prefix_lens, batch, chunk_len, max_len, la.Hkv, la.D, status, s);
+    if (e == cudaSuccess && kt_cache)
+      e = gattn::launch_key_append_transformed(reinterpret_cast<const __nv_bfloat16*>(k_new_or_null), kc, prefix_lens,
+                                               batch, chunk_len, max_len, la, status, s);
     if (e != cudaSuccess) return fail_cuda(e, "kv append launch");
   }
   const __nv_bfloat16* kt = kc;
@@ -412,9 +457,10 @@ int gattn_prefill_chunk(const gattn_bf16* q, const gattn_bf16* k_new_or_null, co
     __nv_bfloat16* qtw = reinterpret_cast<__nv_bfloat16*>(
         ws + round_up(kStatusBytes, 1024) +
         round_up(static_cast<size_t>(batch) * max_len * la.Hkv * la.D * sizeof(uint16_t), 1024));
-    cudaError_t e = gattn::launch_qkprep_chunk(qt, kc, prefix_lens, qtw, ktw, batch, chunk_len, max_len, la, status, s);
+    cudaError_t e = gattn::launch_qkprep_chunk(qt, kc, prefix_lens, qtw, ktw, batch, chunk_len, max_len, la, status, s,
+                                               !kt_cache);
     if (e != cudaSuccess) return fail_cuda(e, "query/key prologue launch");
-    kt = ktw;
+    kt = kt_cache ? kc : ktw;
     qt = qtw;
   }
   gattn::PrefillArgs pa;

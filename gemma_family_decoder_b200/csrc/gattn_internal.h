@@ -27,25 +27,31 @@ struct LayerArgs {
   const float* q_norm_w;
   const float* k_norm_w;
   int k_eq_v;
+  int kt_cache;        // caches hold transformed keys: decode kernels skip the key norm and RoPE
 };
 
 // RoPE table: (cos, sin) of p * theta^(-2t/F) for p < max_pos, t < half.
 cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim, int max_pos,
                               cudaStream_t s);
 
-// q~ = RoPE(RMSNorm(q)) for every (b, s, head) row and k~ = RoPE(RMSNorm(k))
-// for every (b, s, kv head) row, bf16 out, same layouts, in one launch.
-// The chunk form: queries of a chunk (token prefix[b] + i, q only) into qt, and cache
-// keys (token j, rows j < prefix[b] + C only) into kt.
+// The chunk form of launch_qkprep (below): queries of a chunk (token prefix[b] + i,
+// q only) into qt, and cache keys (token j, rows j < prefix[b] + C only) into kt.
 cudaError_t launch_qkprep_chunk(const __nv_bfloat16* q, const __nv_bfloat16* k_cache, const int* prefix,
                                 __nv_bfloat16* qt, __nv_bfloat16* kt, int B, int C, int max_len,
-                                const LayerArgs& la, uint32_t* status, cudaStream_t s);
+                                const LayerArgs& la, uint32_t* status, cudaStream_t s, bool with_keys);
 // Copy a chunk's new rows [B][C][Hkv][D] into cache rows [prefix[b], prefix[b] + C)
 // (v_new / v_cache null when keys and values are tied); a prefix outside
 // [0, max_len - C] is clamped and flagged.
 cudaError_t launch_kv_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new, __nv_bfloat16* k_cache,
                              __nv_bfloat16* v_cache, const int* prefix, int B, int C, int max_len, int Hkv,
                              int D, uint32_t* status, cudaStream_t s);
+// A chunk's new keys [B][C][Hkv][D] transformed at positions prefix[b] + s and
+// written to cache rows prefix[b] + s (a transformed cache's append).
+cudaError_t launch_key_append_transformed(const __nv_bfloat16* k_new, __nv_bfloat16* k_cache, const int* prefix,
+                                          int B, int C, int max_len, const LayerArgs& la, uint32_t* status,
+                                          cudaStream_t s);
+// q~ = RoPE(RMSNorm(q)) for every (b, s, head) row and k~ = RoPE(RMSNorm(k))
+// for every (b, s, kv head) row, bf16 out, same layouts, in one launch.
 cudaError_t launch_qkprep(const __nv_bfloat16* q, const __nv_bfloat16* k, const int* positions,
                           __nv_bfloat16* qt, __nv_bfloat16* kt, int B, int S, const LayerArgs& la,
                           uint32_t* status, cudaStream_t s);

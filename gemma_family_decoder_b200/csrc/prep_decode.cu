@@ -56,7 +56,9 @@ cudaError_t launch_rope_table(float2* tab, double theta, int half, int freq_dim,
 // MODE 0: a prompt's queries and keys, positions from `positions`.  MODE 1: a
 // chunk's queries only (token bs = b * C + s at position prefix[b] + s).
 // MODE 2: a cache's keys only (token bs = b * max_len + s at position s),
-// skipping the rows past the chunk (s >= prefix[b] + C).
+// skipping the rows past the chunk (s >= prefix[b] + C).  MODE 3: a chunk's new
+// keys only (token bs = b * C + s at position prefix[b] + s), written to cache
+// row prefix[b] + s of kt (a transformed cache's append).
 struct ChunkPrep {
   const int* prefix;
   int C, max_len;
@@ -75,14 +77,16 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
   const int i = static_cast<int>(gid % TPR);
   if (bs >= tokens) return;  // whole groups leave together (TPR divides 32)
   int tok_pos = 0;
+  long long kdst = bs;  // output row (token) of the key rows
   if constexpr (MODE == 0) {
     tok_pos = positions ? __ldg(positions + bs) : 0;
   } else {
-    const int per = MODE == 1 ? cp.C : cp.max_len;
+    const int per = MODE == 2 ? cp.max_len : cp.C;
     const int b = static_cast<int>(bs / per), s = static_cast<int>(bs % per);
     const int pre = min(max(__ldg(cp.prefix + b), 0), cp.max_len - cp.C);
     if (MODE == 2 && s >= pre + cp.C) return;  // a cache row no query of the chunk sees
-    tok_pos = MODE == 1 ? pre + s : s;
+    tok_pos = MODE == 2 ? s : pre + s;
+    if (MODE == 3) kdst = static_cast<long long>(b) * cp.max_len + pre + s;
   }
   const unsigned gmask = TPR == 32 ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
   const int h8 = la.rot >> 4;  // chunks in half the rotated slice
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
     for (int e = 0; e < 4; ++e) cs[e] = __ldg(trow + e);
   }
   const float off = la.qk_norm == 1 ? 1.f : 0.f;
-  const int nq = MODE == 2 ? 0 : la.H;  // query rows of the token, then key rows
+  const int nq = MODE >= 2 ? 0 : la.H;  // query rows of the token, then key rows
   const int nrows = nq + (MODE == 1 ? 0 : la.Hkv);
   for (int r0 = 0; r0 < nrows; r0 += RB) {
     uint4 u0[RB], u1[RB];
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(256) qkprep_kernel(const bf16* __restrict__ q,
           x1[e + 1] = b2 * c.z + a2 * c.w;
         }
       }
-      uint4* dst = reinterpret_cast<uint4*>(is_q ? qt + (bs * la.H + r) * D : kt + (bs * la.Hkv + (r - nq)) * D);
+      uint4* dst = reinterpret_cast<uint4*>(is_q ? qt + (bs * la.H + r) * D : kt + (kdst * la.Hkv + (r - nq)) * D);
       dst[c0] = pack8(x0);
       dst[c1] = pack8(x1);
     }
@@ -167,18 +171,30 @@ cudaError_t launch_qkprep(const bf16* q, const bf16* k, const int* positions, bf
 
 cudaError_t launch_qkprep_chunk(const bf16* q, const bf16* k_cache, const int* prefix, bf16* qt, bf16* kt,
                                 int B, int C, int max_len, const LayerArgs& la, uint32_t* status,
-                                cudaStream_t s) {
+                                cudaStream_t s, bool with_keys) {
   const ChunkPrep cp{prefix, C, max_len};
   const long long tq = static_cast<long long>(B) * C, tk = static_cast<long long>(B) * max_len;
   const unsigned bq = static_cast<unsigned>((tq * (la.D / 16) + 255) / 256);
   const unsigned bk = static_cast<unsigned>((tk * (la.D / 16) + 255) / 256);
   if (la.D == 256) {
-    qkprep_kernel<16, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
+    if (with_keys) qkprep_kernel<16, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
     qkprep_kernel<16, 3, 1><<<bq, 256, 0, s>>>(q, nullptr, nullptr, qt, nullptr, tq, la, status, cp);
   } else {
-    qkprep_kernel<32, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
+    if (with_keys) qkprep_kernel<32, 3, 2><<<bk, 256, 0, s>>>(nullptr, k_cache, nullptr, nullptr, kt, tk, la, status, cp);
     qkprep_kernel<32, 3, 1><<<bq, 256, 0, s>>>(q, nullptr, nullptr, qt, nullptr, tq, la, status, cp);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_append_transformed(const bf16* k_new, bf16* k_cache, const int* prefix, int B, int C,
+                                          int max_len, const LayerArgs& la, uint32_t* status, cudaStream_t s) {
+  const ChunkPrep cp{prefix, C, max_len};
+  const long long tk = static_cast<long long>(B) * C;
+  const unsigned bk = static_cast<unsigned>((tk * (la.D / 16) + 255) / 256);
+  if (la.D == 256)
+    qkprep_kernel<16, 3, 3><<<bk, 256, 0, s>>>(nullptr, k_new, nullptr, nullptr, k_cache, tk, la, status, cp);
+  else
+    qkprep_kernel<32, 3, 3><<<bk, 256, 0, s>>>(nullptr, k_new, nullptr, nullptr, k_cache, tk, la, status, cp);
   return cudaGetLastError();
 }
 
@@ -193,13 +209,14 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict_
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gid >= words) return;
   const long long per_b = static_cast<long long>(C) * row_words;  // words of one sequence's new rows
+  // (k_new null: values only, the keys being written transformed by the prologue kernel)
   const int b = static_cast<int>(gid / per_b);
   const long long w = gid % per_b;
   const int raw = __ldg(prefix + b);
   const int pre = min(max(raw, 0), max_len - C);
   if (w == 0 && pre != raw && status) flag_status(status, kStatusBounds);
   const long long dst = (static_cast<long long>(b) * max_len + pre) * row_words + w;
-  k_cache[dst] = __ldg(k_new + gid);
+  if (k_new) k_cache[dst] = __ldg(k_new + gid);
   if (v_new) v_cache[dst] = __ldg(v_new + gid);
 }
 
@@ -300,7 +317,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(DecodeA
     for (int i = 0; i < NCH; ++i)
 #pragma unroll
       for (int e = 0; e < 8; ++e) kx[i][e] = kr[i][e];
-    transform_row<NCH>(kx, lane, j, la, la.k_norm_w, da.status);
+    if (!la.kt_cache) transform_row<NCH>(kx, lane, j, la, la.k_norm_w, da.status);
     float s[HPW];
 #pragma unroll
     for (int hh = 0; hh < HPW; ++hh) {

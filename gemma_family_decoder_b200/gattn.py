@@ -28,7 +28,8 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_prefill", "gattn_decode_workspace_size", "gattn_decode", "gattn_check",
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
            "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded", "gattn_kv_quantize",
-           "gattn_decode_int8", "gattn_prefill_chunk_workspace_size", "gattn_prefill_chunk", "gattn_kv_append")
+           "gattn_decode_int8", "gattn_prefill_chunk_workspace_size", "gattn_prefill_chunk", "gattn_kv_append",
+           "gattn_kv_append_layer")
 
 
 class GattnError(RuntimeError):
@@ -56,6 +57,7 @@ class GattnCfg(ctypes.Structure):
         ("norm_eps", ctypes.c_float),
         ("q_norm_w", ctypes.c_void_p),
         ("k_norm_w", ctypes.c_void_p),
+        ("keys_transformed", ctypes.c_int32),
     ]
 
 
@@ -106,6 +108,8 @@ def lib() -> ctypes.CDLL:
         L.gattn_prefill_chunk.restype = ctypes.c_int
         L.gattn_prefill_chunk.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.POINTER(GattnCfg), vp, sz,
                                           vp]
+        L.gattn_kv_append_layer.restype = ctypes.c_int
+        L.gattn_kv_append_layer.argtypes = [ctypes.POINTER(GattnCfg), vp, vp, vp, vp, vp, i32, i32, i32, vp, vp]
         L.gattn_kv_append.restype = ctypes.c_int
         L.gattn_kv_append.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
         L.gattn_kv_quantize.restype = ctypes.c_int
@@ -154,6 +158,7 @@ class LayerSpec:
     k_eq_v: bool = False
     qk_norm: int = NORM_NONE
     norm_eps: float = 1e-6
+    keys_transformed: bool = False   # KV caches hold keys after QK-norm and RoPE
 
     @property
     def rot_dim(self) -> int:
@@ -161,7 +166,7 @@ class LayerSpec:
 
     @classmethod
     def of(cls, obj) -> "LayerSpec":
-        return cls(**{f: getattr(obj, f) for f in cls.__dataclass_fields__})
+        return cls(**{f: getattr(obj, f) for f in cls.__dataclass_fields__ if hasattr(obj, f)})
 
 
 def rope_table(theta: float, rot_dim: int, freq_dim: int, max_pos: int, device="cuda",
@@ -196,7 +201,8 @@ class AttentionLayer:
             rope_max_pos=max_pos if R > 0 else 0, softcap=spec.softcap, scalar=spec.scalar,
             k_eq_v=int(spec.k_eq_v), qk_norm=spec.qk_norm, norm_eps=spec.norm_eps,
             q_norm_w=None if self.w_q is None else self.w_q.data_ptr(),
-            k_norm_w=None if self.w_k is None else self.w_k.data_ptr())
+            k_norm_w=None if self.w_k is None else self.w_k.data_ptr(),
+            keys_transformed=int(spec.keys_transformed))
 
     # -- workspaces --------------------------------------------------------------
     def prefill_workspace(self, batch: int, seq_len: int, device="cuda") -> torch.Tensor:
@@ -290,6 +296,20 @@ class AttentionLayer:
                                             _ptr(prefix_lens), _ptr(out), B, C, Lmax, ctypes.byref(self.cfg),
                                             _ptr(ws), ws.numel(), _stream(stream)), "gattn_prefill_chunk")
         return out
+
+    def kv_append(self, k_new, v_new, k_cache, v_cache, cache_lens, status=None, stream=None):
+        """gattn_kv_append_layer: rows [B,n,Hkv,D] into caches [B,Lmax,Hkv,D] at rows
+        [cache_lens[b], +n); keys written transformed when the spec's keys_transformed is set."""
+        _need(k_new, "k_new", torch.bfloat16, 4)
+        _need(k_cache, "k_cache", torch.bfloat16, 4)
+        if v_new is not None:
+            _need(v_new, "v_new", torch.bfloat16, 4)
+            _need(v_cache, "v_cache", torch.bfloat16, 4)
+        _need(cache_lens, "cache_lens", torch.int32, 1)
+        B, n = k_new.shape[0], k_new.shape[1]
+        _raise_if(lib().gattn_kv_append_layer(ctypes.byref(self.cfg), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(cache_lens), B, n, k_cache.shape[1], _ptr(status),
+                                              _stream(stream)), "gattn_kv_append_layer")
 
     def decode_int8(self, q, k_codes, k_scales, v_codes=None, v_scales=None, seq_lens=None, out=None,
                     workspace=None, stream=None):

@@ -88,6 +88,13 @@ typedef struct {
   float norm_eps;           /* RMSNorm epsilon (1e-6 in every Gemma card)       */
   const float* q_norm_w;    /* device fp32 [D], shared by heads; NULL iff NONE  */
   const float* k_norm_w;    /* device fp32 [D]; NULL iff NONE                   */
+  int32_t keys_transformed; /* 0: KV caches hold raw keys.  1: caches hold the
+                               keys after QK-norm and RoPE (each at its own
+                               position), as gattn_kv_append_layer and
+                               gattn_prefill_chunk's append write them; the
+                               decode and chunk calls then skip the key
+                               transforms.  Not with k_eq_v (values need the
+                               raw keys).  gattn_prefill ignores it.            */
 } gattn_cfg;
 
 /* ---- RoPE table ---------------------------------------------------------
@@ -186,10 +193,22 @@ int gattn_kv_append(const gattn_bf16* k_new, const gattn_bf16* v_new_or_null, ga
                     int32_t max_len, int32_t num_kv_heads, int32_t head_dim, void* status_or_null,
                     gattn_stream stream);
 
+/* gattn_kv_append_layer: the append of gattn_kv_append for a layer: with
+ * cfg->keys_transformed the key rows are written after QK-norm and RoPE at their
+ * positions cache_lens[b] + s (the rows a transformed cache holds), the values
+ * raw; otherwise it is gattn_kv_append.  cache_lens out of range are clamped and
+ * flag GATTN_ERR_DEVICE_BOUNDS in status_or_null (a gattn workspace), as are
+ * positions past the RoPE table. */
+int gattn_kv_append_layer(const gattn_cfg* cfg, const gattn_bf16* k_new, const gattn_bf16* v_new_or_null,
+                          gattn_bf16* k_cache, gattn_bf16* v_cache_or_null, const int32_t* cache_lens,
+                          int32_t batch, int32_t n_new, int32_t max_len, void* status_or_null,
+                          gattn_stream stream);
+
 /* ---- decode ----------------------------------------------------------------
  * One decode step: query b (at position seq_lens[b]-1) against cache rows
  * [0, seq_lens[b]) of its own cache.  Caches hold RAW keys/values (before
- * QK-norm and RoPE); cached key j sits at position j.
+ * QK-norm and RoPE), or transformed keys with cfg->keys_transformed; cached key
+ * j sits at position j.
  *   q               [batch][H][D]            bf16
  *   k_cache         [batch][max_len][Hkv][D] bf16
  *   v_cache_or_null [batch][max_len][Hkv][D] bf16; NULL (or == k_cache) when k_eq_v

@@ -29,8 +29,9 @@ def test_header_and_exports_agree():
 
 
 def test_cfg_struct_matches_header_layout():
-    # int32 x4, float x2, int32, (pad), ptr, int32, float x2, int32 x2, float, ptr x2
-    assert ctypes.sizeof(G.GattnCfg) == 80
+    # int32 x4, float x2, int32, (pad), ptr, int32, float x2, int32 x2, float, ptr x2, int32, (pad)
+    assert ctypes.sizeof(G.GattnCfg) == 88
+    assert G.GattnCfg.keys_transformed.offset == 80
     assert G.GattnCfg.rope_table.offset == 32
     assert G.GattnCfg.q_norm_w.offset == 64
 
@@ -70,6 +71,8 @@ INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
     (dict(qk_norm=3), INVALID),
     (dict(qk_norm=1), INVALID),                     # weights missing
     (dict(k_eq_v=2), INVALID),
+    (dict(keys_transformed=2), INVALID),
+    (dict(keys_transformed=1, k_eq_v=1), INVALID),     # tied values need the raw keys
 ])
 def test_prefill_rejects_bad_cfg(over, code):
     assert prefill(cfg(**over)) == code

@@ -87,6 +87,7 @@ class ChunkWorkload:
     seed: int
     gain_mean: float = 0.0
     gain_std: float = 0.1
+    keys_transformed: bool = False   # the cache holds transformed keys
 
 
 @dataclasses.dataclass(frozen=True)
@@ -102,6 +103,8 @@ class DecodeWorkload:
     # the cache held as int8 codes + fp32 row scales (Atlas "Gemma 4" summary: int8 KV
     # caching), quantised from the same bf16 rows
     kv_int8: bool = False
+    # the cache holds the keys after QK-norm and RoPE (written by the library's append)
+    keys_transformed: bool = False
 
     @property
     def max_len(self) -> int:
@@ -171,10 +174,19 @@ GEMMA3_GLOBAL_CHUNK = ChunkWorkload(
     "gemma3_1b_global_b8_chunk1024_prefix7168",
     Layer(window=0, rope_theta=1e6, **_G3), batch=8, prefix=7168, chunk=1024, seed=6)
 
+# the same decode and chunk steps over caches holding transformed keys
+GEMMA4_DECODE_LOCAL_TK = dataclasses.replace(GEMMA4_DECODE_LOCAL, name="gemma4_12b_decode_local_tk_b64",
+                                             keys_transformed=True)
+GEMMA4_DECODE_LOCAL_INT8_TK = dataclasses.replace(GEMMA4_DECODE_LOCAL, name="gemma4_12b_decode_local_int8_tk_b64",
+                                                  kv_int8=True, keys_transformed=True)
+GEMMA3_GLOBAL_CHUNK_TK = dataclasses.replace(GEMMA3_GLOBAL_CHUNK, name="gemma3_1b_global_b8_chunk1024_prefix7168_tk",
+                                             keys_transformed=True)
+
 PREFILL: Dict[str, PrefillWorkload] = {w.name: w for w in (
     GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL, GEMMA3_GLOBAL_LEFTPAD)}
 DECODE: Dict[str, DecodeWorkload] = {w.name: w for w in (
-    GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM, GEMMA4_DECODE_LOCAL_INT8)}
+    GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM, GEMMA4_DECODE_LOCAL_INT8,
+    GEMMA4_DECODE_LOCAL_TK, GEMMA4_DECODE_LOCAL_INT8_TK)}
 
 
 # --- drawing -------------------------------------------------------------------
