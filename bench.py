@@ -581,15 +581,21 @@ def cpu_baseline(name, budget_s=15.0):
         per_row = (time.perf_counter() - t0) / len(pilot)
         n = int(max(8, min(S, budget_s / max(per_row, 1e-6))))
         rows = np.unique(np.linspace(0, S - 1, n).astype(np.int64))
-        t0 = time.perf_counter()
-        _oracle_prefill_rows(wl, d, rows)
-        dt = time.perf_counter() - t0
+        # the pilot's per-row cost carries the per-call key transform, so the strided
+        # sample can finish well inside the budget: repeat it until about two thirds of
+        # the budget is spent (at most 16 passes)
+        dt, reps = 0.0, 0
+        while reps < 16 and (reps == 0 or dt < budget_s * 2 / 3):
+            t0 = time.perf_counter()
+            _oracle_prefill_rows(wl, d, rows)
+            dt += time.perf_counter() - t0
+            reps += 1
         L = wl.layer
-        work = rows_flops(wl, d, rows)
+        work = rows_flops(wl, d, rows) * reps
         return {"value": round(work / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
                 "kind": "oracle",
                 "sample": f"{len(rows)} evenly spaced query rows of {S}, all {wl.batch} sequences and "
-                          f"{L.num_heads} heads ({dt:.1f} s, float64 numpy)"}
+                          f"{L.num_heads} heads, {reps} pass(es) ({dt:.1f} s, float64 numpy)"}
     wl = DECODE_WL[name]
     dq = W.decode_inputs(wl)
     lens = dq["seq_lens"].numpy()

@@ -29,7 +29,7 @@ widened) bf16 input values, in the order the layer applies them:
    caching, Table 3 "+KV"): per-row symmetric codes and an fp32 scale,
    dequantised before step 1 (``kv_quantize``, ``attention_decode_int8``).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 scale = scalar**-0.5; softcap after scaling; norm before RoPE; V is the raw k
 when keys and values are tied; rotated dims are the first R = fraction*D dims,
 paired rotate-half (t, t+R/2) with angle pos * theta**(-2t/F), F = head_dim by
