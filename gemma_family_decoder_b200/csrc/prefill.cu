@@ -554,16 +554,19 @@ static cudaError_t run_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaS
   P.q_off = pa.q_off;
   P.KV_S = kv_rows;
   auto kern = prefill_kernel<D, BN, CAP, MODE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  // the shared-memory opt-in is per device: set it once on each device a call runs on
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
   // one CTA per SM (the shared memory allows no more), each taking items in turn
   const long long items = static_cast<long long>(P.nqt) * pa.B * la.H * P.dv_splits;
   if (items > (1LL << 31) - 1) return cudaErrorInvalidValue;
