@@ -15,6 +15,10 @@ Under torchrun (N>1) every rank runs its own replica of the workload on its own
 GPU (independent problems, no collective on the data path: weak scaling); the
 time is the maximum over ranks.  ``--impl reference`` times the float64 CPU
 oracle instead (rank 0 only), on a bounded sample per step.
+
+``--sweep FILE`` runs every workload (or those of ``--sweep-workloads``) in turn and
+appends each one's JSON line to FILE; workloads FILE already holds for the same arm
+are skipped, so an interrupted sweep resumes where it stopped.
 """
 from __future__ import annotations
 
@@ -718,23 +722,78 @@ def main(argv=None):
     ap.add_argument("--len-hi", type=int, default=0,
                     help="decode: draw sequence lengths up to this (and size the cache for it); for profiling")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--sweep", default="", help="append every workload's JSON line to this file, skipping those "
+                                                  "it already holds (resume)")
+    ap.add_argument("--sweep-workloads", default="", help="comma-separated workloads for --sweep (default: all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        return sweep(args, ap)
+    run_one(args)
+
+
+def sweep_done(path: str, impl: str) -> set:
+    """Workloads whose line for this arm is already in the sweep file (unparsable lines,
+    e.g. one cut short by an interrupted run, do not count)."""
+    done = set()
+    if os.path.exists(path):
+        with open(path) as f:
+            for line in f:
+                try:
+                    rec = json.loads(line)
+                except ValueError:
+                    continue
+                if rec.get("impl", "ours") == impl and "config" in rec:
+                    done.add(rec["config"].get("workload"))
+    return done
+
+
+def sweep(args, ap):
+    names = [n for n in args.sweep_workloads.split(",") if n] or \
+        sorted(PREFILL_WL) + sorted(CHUNK_WL) + sorted(DECODE_WL)
+    known = set(PREFILL_WL) | set(CHUNK_WL) | set(DECODE_WL)
+    for n in names:
+        if n not in known:
+            ap.error(f"unknown workload {n}")
+    done = sweep_done(args.sweep, args.impl)  # read once, so every rank skips the same ones
+    for n in names:
+        if n in done:
+            print(f"sweep: {n} already in {args.sweep}, skipped", file=sys.stderr)
+            continue
+        args.workload = n
+        res = run_one(args, emit=False)
+        if res is not None:
+            line = json.dumps(res)
+            print(line, flush=True)
+            with open(args.sweep, "a+b") as f:  # one write per line, on a fresh line
+                f.seek(0, os.SEEK_END)
+                lead = b""
+                if f.tell() > 0:
+                    f.seek(-1, os.SEEK_END)
+                    lead = b"" if f.read(1) == b"\n" else b"\n"  # after a line cut short
+                f.write(lead + line.encode() + b"\n")
+
+
+def run_one(args, emit=True):
+    """One workload on this arm; rank 0 returns (and by default prints) its JSON line."""
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores only; other ranks have no work
         rank = int(os.environ.get("RANK", "0"))
         res = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
-        if res is not None:
+        if res is not None and emit:
             print(json.dumps(res), flush=True)
-        return
+        return res
     world, rank, local = dist_setup()
     if world != args.gpus and rank == 0:
         print(f"note: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
     try:
         res = run_ours(args, world, rank, local)
-        if rank == 0 and res is not None:
+        if rank != 0:
+            res = None
+        if res is not None and emit:
             print(json.dumps(res), flush=True)
+        return res
     finally:
         import torch.distributed as dist
         if dist.is_available() and dist.is_initialized():

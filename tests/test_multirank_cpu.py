@@ -82,3 +82,33 @@ def test_reference_arm_under_torchrun_prints_once():
     assert res["impl"] == "reference" and res["n_gpus"] == 2 and res["steps"] == 3
     assert res["value"] > 0 and res["e2e"]["h2d_bytes_per_step"] == 0
     assert res["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_sweep_appends_each_workload_once_and_resumes(tmp_path):
+    out = tmp_path / "sweep.jsonl"
+    env = dict(os.environ, GATTN_REF_BUDGET_S="1", OMP_NUM_THREADS="1")
+
+    def run(names):
+        cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3", "--warmup", "3",
+               "--sweep", str(out), "--sweep-workloads", names]
+        r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        return r
+
+    run("gemma2_2b_local_s256,gemma4_12b_decode_local_b64")
+    lines = out.read_text().splitlines()
+    assert [json.loads(ln)["config"]["workload"] for ln in lines] == ["gemma2_2b_local_s256",
+                                                                     "gemma4_12b_decode_local_b64"]
+    # an interrupted run's partial line is ignored; done workloads are skipped
+    with open(out, "a") as f:
+        f.write('{"metric": "cut sho')
+    r = run("gemma2_2b_local_s256,gemma4_12b_decode_local_b64,gemma3_1b_global_b8_chunk1024_prefix7168")
+    assert r.stderr.count("skipped") == 2
+    recs = []
+    for ln in out.read_text().splitlines():
+        try:
+            recs.append(json.loads(ln))
+        except ValueError:
+            pass
+    assert [x["config"]["workload"] for x in recs][-1] == "gemma3_1b_global_b8_chunk1024_prefix7168"
+    assert len(recs) == 3 and all(x["impl"] == "reference" for x in recs)
