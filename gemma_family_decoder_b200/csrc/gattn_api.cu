@@ -522,7 +522,7 @@ static int decode_launch(gattn::DecodeArgs& da, const gattn::LayerArgs& la, cons
   da.trace_bytes = g_trace_buf ? g_trace_bytes : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (g_prof_start) cudaEventRecord(g_prof_start, s);
-  cudaError_t e = da.kq ? gattn::launch_decode_simt(da, la, s) : gattn::launch_decode_split(da, la, s);
+  cudaError_t e = gattn::launch_decode_split(da, la, s);
   if (g_prof_stop) cudaEventRecord(g_prof_stop, s);
   if (e != cudaSuccess) return fail_cuda(e, "decode split launch");
   e = gattn::launch_decode_combine(da, la, s);
@@ -588,9 +588,8 @@ int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k
   gattn::LayerArgs la;
   int st = resolve(cfg, &la, true);
   if (st != GATTN_OK) return st;
-  if (!gattn::decode_simt_supported(la))
-    return fail(GATTN_ERR_UNSUPPORTED,
-                "int8 cache: 1, 2 or 4 query heads per kv head (head_dim 512: 1 or 2) and 1, 2, 4 or 8 kv heads");
+  st = decode_supported(la);
+  if (st != GATTN_OK) return st;
   if (batch < 0 || max_len <= 0) return fail(GATTN_ERR_INVALID_ARG, "batch must be >= 0 and max_len > 0");
   if (!q || !k_codes || !k_scales || !out || !seq_lens)
     return fail(GATTN_ERR_INVALID_ARG, "q, k_codes, k_scales, seq_lens and out must not be NULL");

@@ -33,6 +33,23 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16* row, int lane, flo
   }
 }
 
+// The same chunks from an int8 row, dequantised by the row's scale.
+template <int NCH>
+__device__ __forceinline__ void load_row_q8(const int8_t* row, float scale, int lane, float (&x)[NCH][8]) {
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + lane + 32 * i);
+    float2 c[4];
+    unpack_i8x4(u.x, c[0], c[1]);
+    unpack_i8x4(u.y, c[2], c[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[i][2 * e] = c[e].x * scale;
+      x[i][2 * e + 1] = c[e].y * scale;
+    }
+  }
+}
+
 __device__ __forceinline__ int checked_pos(int pos, const LayerArgs& la, uint32_t* status) {
   if (pos < 0 || pos >= la.rope_max_pos) {
     flag_status(status, kStatusBounds);

@@ -309,9 +309,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(DecodeA
   const float log2e_cap = la.softcap > 0.f ? 1.4426950408889634f : 0.f;
 
   for (int j = start + kg; j < end; j += KW) {
-    const size_t rowoff = ((static_cast<size_t>(b) * da.max_len + j) * la.Hkv + kvh) * D;
+    const size_t rowidx = (static_cast<size_t>(b) * da.max_len + j) * la.Hkv + kvh;  // (position, kv head)
+    const size_t rowoff = rowidx * D;
     float kr[NCH][8];
-    load_row<NCH>(da.k + rowoff, lane, kr);
+    if (da.kq) load_row_q8<NCH>(da.kq + rowoff, __ldg(da.ks + rowidx), lane, kr);  // an int8 cache
+    else load_row<NCH>(da.k + rowoff, lane, kr);
     float kx[NCH][8];
 #pragma unroll
     for (int i = 0; i < NCH; ++i)
@@ -333,7 +335,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(DecodeA
         s[hh] = la.softcap * tanhf(nat / la.softcap) * log2e_cap;
       }
     }
-    if (!la.k_eq_v) load_row<NCH>(da.v + rowoff, lane, kr);
+    if (!la.k_eq_v) {
+      if (da.kq) load_row_q8<NCH>(da.vq + rowoff, __ldg(da.vs + rowidx), lane, kr);
+      else load_row<NCH>(da.v + rowoff, lane, kr);
+    }
 #pragma unroll
     for (int hh = 0; hh < HPW; ++hh) {
       const float mn = fmaxf(m[hh], s[hh]);
@@ -478,7 +483,8 @@ static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, c
 }
 
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
-  if (decode_tc_supported(la)) return launch_decode_tc(da, la, s);
+  // an int8 cache (da.kq): the persistent CUDA-core kernel, else the split kernel below
+  if (!da.kq && decode_tc_supported(la)) return launch_decode_tc(da, la, s);
   if (decode_simt_supported(la)) return launch_decode_simt(da, la, s);
   const int hpw = la.G <= 2 ? la.G : la.G / 4;
   if (la.D == 256) {

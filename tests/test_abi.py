@@ -128,7 +128,7 @@ def decode_int8(c, q=ALIGNED, kc=ALIGNED, ks=ALIGNED, vc=ALIGNED, vs=ALIGNED, le
 
 def test_decode_int8_rejects_bad_args():
     c = cfg(num_heads=16, num_kv_heads=8)
-    assert decode_int8(cfg(num_heads=16, num_kv_heads=1)) == UNSUPPORTED   # 16 per kv head: no int8 kernel
+    assert decode_int8(cfg(num_heads=24, num_kv_heads=1)) == UNSUPPORTED   # group of 24, as gattn_decode
     assert decode_int8(c, kc=None) == INVALID
     assert decode_int8(c, ks=ALIGNED + 2) == INVALID
     assert decode_int8(c, kc=ALIGNED + 4) == INVALID

@@ -1,4 +1,5 @@
-"""GPU parity of the int8 KV cache: gattn_kv_quantize and gattn_decode_int8.
+"""GPU parity of the int8 KV cache: gattn_kv_quantize and gattn_decode_int8 (the persistent
+CUDA-core kernel for 1, 2 or 4 query heads per kv head, the split kernel for 8 or 16).
 
 The quantiser is integer work decided by float32 division on both sides, so
 its codes and scales must equal the oracle's bit for bit.  The int8 decode is
@@ -114,6 +115,12 @@ INT8_CASES = [
                                          k_eq_v=True), [1, 9, 64, 65]),
     ("g2_d256_r16_cap_w5", W.Layer(num_heads=8, num_kv_heads=4, head_dim=256, rotary_fraction=0.0625,
                                    softcap=30.0, window=5), [1, 4, 5, 6, 40]),
+    # 8 or 16 query heads per kv head: the CUDA-core split kernel reading int8 rows
+    ("global_keqv_g16_d512", W.GEMMA4_DECODE_GLOBAL.layer, [1, 700, 2049, 2500]),
+    ("keqv_g8_d512_norm", W.Layer(num_heads=8, num_kv_heads=1, head_dim=512, rope_theta=1e6, rotary_fraction=0.25,
+                                  scalar=512.0, k_eq_v=True, qk_norm=W.NORM_W), [3, 65, 700]),
+    ("g8_d256_window_cap", W.Layer(num_heads=16, num_kv_heads=2, head_dim=256, window=200, softcap=30.0),
+     [1, 199, 200, 201, 900]),
 ]
 
 
