@@ -207,3 +207,11 @@ def test_status_strings():
     for code in range(7):
         assert L.gattn_status_string(code)
     assert G.version().startswith("libgattn")
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback of any kind: without libgattn.so every call raises
+    monkeypatch.setattr(gattn, "_lib", None)
+    monkeypatch.setattr(gattn, "LIB_PATH", str(tmp_path / "absent" / "libgattn.so"))
+    with pytest.raises(ImportError):
+        gattn.lib()
