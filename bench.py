@@ -51,7 +51,8 @@ PREFILL_WL = {
 }
 DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
                                  W.GEMMA4_DECODE_GLOBAL_NORM, W.GEMMA4_DECODE_LOCAL_INT8,
-                                 W.GEMMA4_DECODE_LOCAL_TK, W.GEMMA4_DECODE_LOCAL_INT8_TK)}
+                                 W.GEMMA4_DECODE_LOCAL_TK, W.GEMMA4_DECODE_LOCAL_INT8_TK,
+                                 W.GEMMA4_DECODE_GLOBAL_INT8)}
 CHUNK_WL = {w.name: w for w in (W.GEMMA3_GLOBAL_CHUNK, W.GEMMA3_GLOBAL_CHUNK_TK)}
 HEADLINE = "gemma1_2b_mqa_b4_s2048"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -296,12 +297,12 @@ def make_chunk(wl, dev):
                             "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 
-def dominant_decode_src(L: W.Layer) -> str:
+def dominant_decode_src(L: W.Layer, int8: bool = False) -> str:
     """Source of the split kernel a decode layer runs (the step's dominant kernel): the
-    tensor-core one for K=V with 8 or 16 query heads per kv head, the CUDA-core one for
-    1, 2 or 4, else the fallback in the prologue/combine file."""
+    tensor-core one for K=V with 8 or 16 query heads per kv head (bf16 caches), the
+    CUDA-core one for 1, 2 or 4, else the split kernel in the prologue/combine file."""
     G = L.num_heads // L.num_kv_heads
-    if L.k_eq_v and G in (8, 16):
+    if L.k_eq_v and G in (8, 16) and not int8:
         return "gemma_family_decoder_b200/csrc/decode_tc.cu"
     if G in (1, 2, 4):
         return "gemma_family_decoder_b200/csrc/decode_simt.cu"
@@ -359,7 +360,7 @@ def make_decode(wl, dev):
     return dict(layer=layer, host=host, dev=devt, out=out, host_out=host_out, ws=ws, step=step,
                 work=decode_bytes(L, lens.numpy(), wl.kv_int8), unit="GB/s", scale=1e9,
                 metric="decode KV GB/s (algorithmic bytes)", bound="hbm", launches=2,
-                kernel_src=(dominant_decode_src(L), "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
+                kernel_src=(dominant_decode_src(L, wl.kv_int8), "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 
 def run_ours(args, world, rank, local):

@@ -174,6 +174,9 @@ GEMMA3_GLOBAL_CHUNK = ChunkWorkload(
     "gemma3_1b_global_b8_chunk1024_prefix7168",
     Layer(window=0, rope_theta=1e6, **_G3), batch=8, prefix=7168, chunk=1024, seed=6)
 
+# the global K=V decode over an int8 cache (the CUDA-core split kernel)
+GEMMA4_DECODE_GLOBAL_INT8 = dataclasses.replace(GEMMA4_DECODE_GLOBAL, name="gemma4_12b_decode_global_keqv_int8_b64",
+                                                kv_int8=True)
 # the same decode and chunk steps over caches holding transformed keys
 GEMMA4_DECODE_LOCAL_TK = dataclasses.replace(GEMMA4_DECODE_LOCAL, name="gemma4_12b_decode_local_tk_b64",
                                              keys_transformed=True)
@@ -186,7 +189,7 @@ PREFILL: Dict[str, PrefillWorkload] = {w.name: w for w in (
     GEMMA2_LOCAL, GEMMA1_MQA, GEMMA3_LOCAL, GEMMA3_GLOBAL, GEMMA4_GLOBAL, GEMMA3_GLOBAL_LEFTPAD)}
 DECODE: Dict[str, DecodeWorkload] = {w.name: w for w in (
     GEMMA4_DECODE_LOCAL, GEMMA4_DECODE_GLOBAL, GEMMA4_DECODE_GLOBAL_NORM, GEMMA4_DECODE_LOCAL_INT8,
-    GEMMA4_DECODE_LOCAL_TK, GEMMA4_DECODE_LOCAL_INT8_TK)}
+    GEMMA4_DECODE_LOCAL_TK, GEMMA4_DECODE_LOCAL_INT8_TK, GEMMA4_DECODE_GLOBAL_INT8)}
 
 
 # --- drawing -------------------------------------------------------------------
