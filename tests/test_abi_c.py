@@ -32,7 +32,7 @@ def test_c_client_layout_and_host_calls(tmp_path):
     assert r.returncode == 0, r.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, run.stderr
-    out = dict(line.rsplit(" ", 1) for line in run.stdout.strip().splitlines())
+    out = dict(line.split("=", 1) for line in run.stdout.strip().splitlines())
     assert int(out["sizeof"]) == ctypes.sizeof(G.GattnCfg)
     for field in ("rope_table", "q_norm_w", "keys_transformed"):
         assert int(out[f"offset {field}"]) == getattr(G.GattnCfg, field).offset, field
