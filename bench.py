@@ -3,13 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Default workload: the Gemma-1-2b-shaped global MQA prefill (batch 4, seq 2048,
-8 query heads, 1 KV head, head_dim 256, full causal, RoPE theta 1e4), metric
-"attention prefill TFLOP/s" on effective (visible-pair) FLOPs.  A step is one
-gattn_prefill call (key prologue + tensor-core attention kernel) on inputs
-already resident in HBM; L2 is flushed (256 MiB write) before every step and
-the flush is outside the per-step CUDA-event timing.  Decode workloads report
-KV GB/s on algorithmic bytes.
+Default workload: the largest single-GPU configuration, the Gemma-4-12b-shaped
+global K=V prefill (batch 1, seq 32768, 16 query heads, 1 KV head, head_dim 512,
+partial RoPE 0.25, plain-weight QK-norm, full causal), metric "attention prefill
+TFLOP/s" on effective (visible-pair) FLOPs.  A step is one gattn_prefill call
+(query/key prologue + tensor-core attention kernel) on inputs already resident
+in HBM; L2 is flushed (256 MiB write) before every step and the flush is outside
+the per-step CUDA-event timing.  Decode workloads report KV GB/s on algorithmic
+bytes; the default line also carries both Gemma-4 decode layers (local and
+global K=V, batch 64), each timed the same way, under "decode".
 
 Under torchrun (N>1) every rank runs its own replica of the workload on its own
 GPU (independent problems, no collective on the data path: weak scaling); the
@@ -54,7 +56,9 @@ DECODE_WL = {w.name: w for w in (W.GEMMA4_DECODE_LOCAL, W.GEMMA4_DECODE_GLOBAL,
                                  W.GEMMA4_DECODE_LOCAL_TK, W.GEMMA4_DECODE_LOCAL_INT8_TK,
                                  W.GEMMA4_DECODE_GLOBAL_INT8)}
 CHUNK_WL = {w.name: w for w in (W.GEMMA3_GLOBAL_CHUNK, W.GEMMA3_GLOBAL_CHUNK_TK)}
-HEADLINE = "gemma1_2b_mqa_b4_s2048"
+HEADLINE = "gemma4_12b_global_keqv_s32768"
+# decode layers measured alongside the headline prefill (their own timed steps)
+HEADLINE_DECODE = ("gemma4_12b_decode_local_b64", "gemma4_12b_decode_global_keqv_b64")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -258,9 +262,18 @@ def make_prefill(wl, dev):
                 work=prefill_flops(wl, d["seq_range"]), unit="TFLOP/s", scale=1e12,
                 metric="attention prefill TFLOP/s (effective FLOPs)", bound="tensor",
                 launches=2 if (wl.layer.rot_dim or wl.layer.qk_norm) else 1,
-                kernel_src=("gemma_family_decoder_b200/csrc/prefill.cu",
+                kernel_src=(dominant_prefill_src(wl.layer, d["seq_range"] is not None),
                             "gemma_family_decoder_b200/csrc/kernels/common.cuh"),
                 oracle=lambda: d)
+
+
+def dominant_prefill_src(L: W.Layer, padded: bool) -> str:
+    """Source of the attention kernel a whole-prompt prefill runs: the SM-pair kernel for
+    head_dim 512 with an even number of query heads per kv head, else the single-SM one."""
+    G = L.num_heads // L.num_kv_heads
+    if L.head_dim == 512 and G % 2 == 0 and not padded:
+        return "gemma_family_decoder_b200/csrc/prefill_pair.cu"
+    return "gemma_family_decoder_b200/csrc/prefill.cu"
 
 
 def make_chunk(wl, dev):
@@ -363,11 +376,7 @@ def make_decode(wl, dev):
                 kernel_src=(dominant_decode_src(L, wl.kv_int8), "gemma_family_decoder_b200/csrc/kernels/common.cuh"))
 
 
-def run_ours(args, world, rank, local):
-    from gemma_family_decoder_b200 import check, set_profile_events
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    name = args.workload
+def make_runner(name, args, dev):
     is_prefill = name in PREFILL_WL
     is_chunk = name in CHUNK_WL
     wl = PREFILL_WL[name] if is_prefill else CHUNK_WL[name] if is_chunk else DECODE_WL[name]
@@ -376,32 +385,39 @@ def run_ours(args, world, rank, local):
         # shortest sequence the work per step is the same
         wl = dataclasses.replace(wl, len_hi=max(wl.len_lo, args.len_hi))
     R = make_prefill(wl, dev) if is_prefill else make_chunk(wl, dev) if is_chunk else make_decode(wl, dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    flush_r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty((), dtype=torch.float32, device=dev)
+    R.update(wl=wl, is_prefill=is_prefill, is_chunk=is_chunk)
+    return R
+
+
+class L2Flush:
+    """A write larger than L2 evicts the inputs; the read that follows drains the
+    write's dirty lines, so that their write-back to HBM does not overlap the timed step."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
+def time_steps(R, args, dev, flush, K):
+    """W warm-up steps, then K timed steps (each one CUDA-graph replay of the library
+    call, L2 flushed before each outside its events), then the main kernel's own time on
+    eager calls from the library's profile events around its launch.  Returns the per-step
+    times, the kernel times, the clock summary and the wall time of the timed loop."""
+    from gemma_family_decoder_b200 import check, set_profile_events
     stream = torch.cuda.current_stream()
-
-    def flush_l2():
-        # a write larger than L2 evicts the inputs; the read that follows
-        # drains the write's dirty lines, so that their write-back to HBM does
-        # not overlap the timed step
-        flush.zero_()
-        torch.sum(flush_r, dim=0, out=sink)
-
     for _ in range(args.warmup):
-        flush_l2()
+        flush()
         R["step"]()
     torch.cuda.synchronize()
     st = check(R["ws"])
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
-
-    K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    # The timed step is one replay of a CUDA graph of the library call (all of
-    # its launches), so that host-side call overhead cannot open gaps inside
-    # the step.  The main kernel's own time is taken afterwards on eager calls,
-    # from the library's profile events around that kernel's launch.
     kev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     for e in kev:  # torch creates the CUDA event at its first record; the library re-records it
         e.record(stream)
@@ -419,7 +435,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for i in range(K):
-        flush_l2()
+        flush()
         ev[i][0].record(stream)
         if graph is not None:
             graph.replay()
@@ -436,12 +452,41 @@ def run_ours(args, world, rank, local):
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
     kern_ms = []
     for i in range(min(K, 200)):
-        flush_l2()
+        flush()
         set_profile_events(kev[0], kev[1])
         R["step"]()
         set_profile_events(None, None)
         torch.cuda.synchronize()
         kern_ms.append(kev[0].elapsed_time(kev[1]))
+    del graph
+    return step_ms, kern_ms, sampler.summary(), wall
+
+
+def roofline(R, name, kern_mean):
+    peaks, peak_src = load_peaks()
+    achieved = R["work"] / (kern_mean / 1e3) / R["scale"]
+    if R["bound"] == "tensor":
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        peak_unit = "TFLOP/s"
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        peak_unit = "GB/s"
+    return {"bound": R["bound"], "achieved": round(achieved, 3), "peak": peak,
+            "unit": peak_unit, "frac": round(achieved / peak, 4), "traffic": profiled_traffic(name, R["kernel_src"]),
+            "peak_source": f"{peak_src} ({'bf16_tflops burst' if R['bound'] == 'tensor' else 'hbm_gbs copy'})",
+            "kernel_ms": round(kern_mean, 5)}
+
+
+def run_ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    name = args.workload
+    R = make_runner(name, args, dev)
+    wl, is_prefill, is_chunk = R["wl"], R["is_prefill"], R["is_chunk"]
+    flush = L2Flush(dev)
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    step_ms, kern_ms, clocks, wall = time_steps(R, args, dev, flush, K)
     total_ms = reduce_max(sum(step_ms), dev)
 
     # end to end through the public call: pinned host inputs in, result out, every step
@@ -462,19 +507,10 @@ def run_ours(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev) / E
+    del scratch
 
-    peaks, peak_src = load_peaks()
     unit, scale = R["unit"], R["scale"]
     value = R["work"] * world * K / (total_ms / 1e3) / scale
-    kern_mean = statistics.mean(kern_ms)
-    achieved = R["work"] / (kern_mean / 1e3) / scale
-    if R["bound"] == "tensor":
-        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-        peak_unit = "TFLOP/s"
-    else:
-        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        peak_unit = "GB/s"
-    traffic = profiled_traffic(name, R["kernel_src"])
     result = {
         "metric": R["metric"], "value": round(value, 3), "unit": unit, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
@@ -482,19 +518,32 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": name, "l2": "flushed before every step (256 MiB write, then a 256 MiB read "
                    "that drains the write's dirty lines), outside the per-step CUDA-event time",
-                   "step": "eager library call" if graph is None else "CUDA-graph replay of the library call",
+                   "step": "eager library call" if args.eager else "CUDA-graph replay of the library call",
                    **({"len_hi": wl.len_hi} if args.len_hi and not is_prefill and not is_chunk else {}),
                    "parallelism": f"replicas{world}"},
-        "roofline": {"bound": R["bound"], "achieved": round(achieved, 3), "peak": peak,
-                     "unit": peak_unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if R['bound'] == 'tensor' else 'hbm_gbs copy'})",
-                     "kernel_ms": round(kern_mean, 5)},
+        "roofline": roofline(R, name, statistics.mean(kern_ms)),
         "e2e": {"value": round(R["work"] * world / (e2e_ms / 1e3) / scale, 3), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": R["launches"] * K,
-        "clocks": sampler.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": round(wall, 3),
     }
+    del R
+    torch.cuda.empty_cache()
+    if name == HEADLINE and not args.no_decode:
+        # the decode target is measured in the same run: each layer its own timed steps
+        result["decode"] = []
+        for dn in HEADLINE_DECODE:
+            D = make_runner(dn, args, dev)
+            d_steps, d_kern, d_clocks, _ = time_steps(D, args, dev, flush, K)
+            d_total = reduce_max(sum(d_steps), dev)
+            result["decode"].append({
+                "workload": dn, "metric": D["metric"],
+                "value": round(D["work"] * world * K / (d_total / 1e3) / D["scale"], 3), "unit": D["unit"],
+                "ms_per_step": round(d_total / K, 5), "roofline": roofline(D, dn, statistics.mean(d_kern)),
+                "gpu_launches": D["launches"] * K, "clocks": d_clocks})
+            del D
+            torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(name, budget_s=args.cpu_budget)
     return result
@@ -719,6 +768,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(PREFILL_WL) + sorted(CHUNK_WL) + sorted(DECODE_WL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode layers measured with the headline")
     ap.add_argument("--eager", action="store_true", help="time eager library calls instead of a graph replay")
     ap.add_argument("--len-hi", type=int, default=0,
                     help="decode: draw sequence lengths up to this (and size the cache for it); for profiling")

@@ -117,6 +117,12 @@ struct PrefillArgs {
 };
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
 
+// Head_dim 512 prefill on SM pairs (tcgen05 cta_group::2; see
+// prefill_pair.cu): whole prompts of layers with an even number of query heads
+// per kv head.  Same arguments as launch_prefill.
+bool prefill_pair_supported(const LayerArgs& la);
+cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s);
+
 // Self-test: one CTA waits on an mbarrier nobody arrives on.
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t timeout_ns, cudaStream_t s);
 

@@ -587,6 +587,8 @@ static cudaError_t launch_prefill_mode(const PrefillArgs& pa, const LayerArgs& l
 cudaError_t launch_prefill(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
   if (pa.seq_range) return launch_prefill_mode<1>(pa, la, s);
   if (pa.q_off) return launch_prefill_mode<2>(pa, la, s);
+  // whole prompts at head_dim 512: two heads of a kv group on an SM pair
+  if (prefill_pair_supported(la)) return launch_prefill_pair(pa, la, s);
   return launch_prefill_mode<0>(pa, la, s);
 }
 

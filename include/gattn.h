@@ -146,7 +146,9 @@ int gattn_prefill(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_
  * rows of padding tokens are zero.  Positions of padding tokens must still be
  * in [0, rope_max_pos) (they are rotated, then ignored).  Every other argument,
  * the workspace size and the errors are those of gattn_prefill; with every
- * range [0, seq_len) the result is bit-identical to gattn_prefill's.  Padding
+ * range [0, seq_len) the result is bit-identical to gattn_prefill's, except on
+ * head_dim-512 layers with an even number of query heads per kv head, whose
+ * whole prompts run on SM pairs (equal within rounding there).  Padding
  * rows of k and v get weight exactly 0 but are read: they must be finite. */
 int gattn_prefill_padded(const gattn_bf16* q, const gattn_bf16* k, const gattn_bf16* v_or_null,
                          const int32_t* positions, const int32_t* seq_range, gattn_bf16* out,

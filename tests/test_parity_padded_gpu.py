@@ -94,8 +94,12 @@ def test_padded_prefill_matches_oracle(name, over, S, ranges):
     check_padding_rows_zero(out, ranges)
 
 
+# head_dim 512 with an odd number of query heads per kv head: whole prompts and
+# padded batches run the same single-SM kernel (even groups take the SM-pair
+# kernel for whole prompts, equal to the padded path within rounding:
+# test_parity_pair_gpu.py)
 @pytest.mark.parametrize("over,S", [(dict(), 300), (dict(window=128), 257),
-                                    (dict(head_dim=512, num_heads=2, num_kv_heads=1, scalar=512.0), 130)])
+                                    (dict(head_dim=512, num_heads=3, num_kv_heads=1, scalar=512.0), 130)])
 def test_full_ranges_bit_identical_to_unpadded(over, S):
     layer = W.Layer(**{**BASE, **over})
     d = small_prefill_inputs(layer, 2, S, seed=41)
