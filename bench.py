@@ -384,6 +384,9 @@ def make_runner(name, args, dev):
         # a smaller cache for profiling; with a window no longer than the
         # shortest sequence the work per step is the same
         wl = dataclasses.replace(wl, len_hi=max(wl.len_lo, args.len_hi))
+    if args.seq and is_prefill:
+        # a shorter prompt of the same layer, for profiling captures
+        wl = dataclasses.replace(wl, seq=args.seq)
     R = make_prefill(wl, dev) if is_prefill else make_chunk(wl, dev) if is_chunk else make_decode(wl, dev)
     R.update(wl=wl, is_prefill=is_prefill, is_chunk=is_chunk)
     return R
@@ -520,6 +523,7 @@ def run_ours(args, world, rank, local):
                    "that drains the write's dirty lines), outside the per-step CUDA-event time",
                    "step": "eager library call" if args.eager else "CUDA-graph replay of the library call",
                    **({"len_hi": wl.len_hi} if args.len_hi and not is_prefill and not is_chunk else {}),
+                   **({"seq": wl.seq} if args.seq and is_prefill else {}),
                    "parallelism": f"replicas{world}"},
         "roofline": roofline(R, name, statistics.mean(kern_ms)),
         "e2e": {"value": round(R["work"] * world / (e2e_ms / 1e3) / scale, 3), "unit": unit,
@@ -530,7 +534,7 @@ def run_ours(args, world, rank, local):
     }
     del R
     torch.cuda.empty_cache()
-    if name == HEADLINE and not args.no_decode:
+    if name == HEADLINE and not (args.no_decode or args.seq):
         # the decode target is measured in the same run: each layer its own timed steps
         result["decode"] = []
         for dn in HEADLINE_DECODE:
@@ -772,6 +776,8 @@ def main(argv=None):
     ap.add_argument("--eager", action="store_true", help="time eager library calls instead of a graph replay")
     ap.add_argument("--len-hi", type=int, default=0,
                     help="decode: draw sequence lengths up to this (and size the cache for it); for profiling")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="prefill: a prompt of this many tokens instead of the workload's; for profiling")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--sweep", default="", help="append every workload's JSON line to this file, skipping those "
                                                   "it already holds (resume)")

@@ -393,8 +393,11 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr)
                : "memory");
 }
+// Expect `bytes` of asynchronous copies on an mbarrier of any CTA of the
+// cluster and arrive on it; relaxed: the arriving thread orders no data of its
+// own (the copies' bytes complete the phase), so no cluster-wide fence.
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_cluster_addr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
                    bar_cluster_addr),
                "r"(bytes)
                : "memory");

@@ -101,12 +101,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* full = bars;                    // [NUNIT] first CTA: both CTAs' bytes of a unit
   uint64_t* empty = bars + C::NUNIT;        // [NUNIT] both CTAs: the unit's MMAs are done
   uint64_t* s_full = bars + 2 * C::NUNIT;   // [2] both: S ready in its TMEM slot
-  uint64_t* p_full = s_full + 2;            // [2] first CTA: P written (256 arrivals)
+  uint64_t* p_full = s_full + 2;            // [2] first CTA: P written (one arrival per softmax warp)
   uint64_t* o_done = p_full + 2;            // both: one phase per P V
   uint64_t* q_full = o_done + 1;            // first CTA: both Q tiles landed
   uint64_t* q_empty = q_full + 1;           // both: the item's last Q K^T is done
   uint64_t* o_final = q_empty + 1;          // both: the item's last P V is done
-  uint64_t* o_empty = o_final + 1;          // first CTA: both softmaxes read O (256 arrivals)
+  uint64_t* o_empty = o_final + 1;          // first CTA: both softmaxes read O (one arrival per warp)
   uint64_t* drain = o_empty + 1;            // first CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -155,13 +155,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
+      mbar_init(&p_full[i], 8);
     }
     mbar_init(o_done, 1);
     mbar_init(q_full, 2);
     mbar_init(q_empty, 1);
     mbar_init(o_final, 1);
-    mbar_init(o_empty, 256);
+    mbar_init(o_empty, 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -310,7 +310,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         l = (rescale ? l * alpha : l) + rs;
         m = m_use;
         tc_fence_before();
-        mbar_arrive_cluster(p_full_l[T & 1]);
+        // the warp's tensor-memory stores are complete (wait::st is warp-wide):
+        // one cluster-scope arrival per warp instead of one fence per thread
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full_l[T & 1]);
         if (t == 0 && I == 0 && j < 120) mark(128 + j);
       }
       ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, I & 1, tmo, P.status, abort_flag));
@@ -339,7 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive_cluster(o_empty_l);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(o_empty_l);
       T0 += w.ntiles;
       ++I;
     }
