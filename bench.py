@@ -129,15 +129,6 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
 
@@ -606,159 +597,197 @@ def _oracle_chunk(wl, d, rows):
                                      rows=rows)
 
 
-def cpu_baseline(name, budget_s=15.0):
-    """The oracle timed on a strided sample of query rows (prefill) or batch rows (decode)."""
-    import oracle as O
-    if name in CHUNK_WL:
-        wl = CHUNK_WL[name]
-        d = W.chunk_inputs(wl)
-        _oracle_chunk(wl, d, np.array([0]))  # warm-up
-        # rows cost little next to each call's key transform: grow the strided sample
-        # until it takes about a quarter of the budget (or is the whole chunk)
-        n = 16
-        while True:
-            rows = np.unique(np.linspace(0, wl.chunk - 1, n).astype(np.int64))
-            t0 = time.perf_counter()
-            _oracle_chunk(wl, d, rows)
-            dt = time.perf_counter() - t0
-            if n >= wl.chunk or dt > budget_s / 4:
-                break
-            n = min(wl.chunk, n * 4)
-        return {"value": round(chunk_flops(wl, rows) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
-                "kind": "oracle",
-                "sample": f"{len(rows)} evenly spaced chunk rows of {wl.chunk}, all {wl.batch} sequences and "
-                          f"{wl.layer.num_heads} heads ({dt:.1f} s, float64 numpy)"}
-    if name in PREFILL_WL:
-        wl = PREFILL_WL[name]
-        d = W.prefill_inputs(wl)
-        S = wl.seq
-        pilot = np.arange(0, S, max(1, S // 8))
-        _oracle_prefill_rows(wl, d, pilot[:2])  # first call: library and cache warm-up
+# The oracle runs in a process pool over independent units (query-row blocks of a
+# prompt, batch rows of a decode step) on the host's cores, one BLAS thread per
+# worker.  Workers are started with "spawn" (never fork a process that has
+# touched CUDA) and get the inputs through torch shared memory; the pool size is
+# the core count, capped by the host memory the float64 oracle needs per worker.
+
+_POOL = {}
+
+
+def _pool_init(kind, name, data):
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:
+        pass
+    torch.set_num_threads(1)
+    _POOL.update(kind=kind, name=name, data=data)
+
+
+def _pool_task(arg):
+    kind, name, data = _POOL["kind"], _POOL["name"], _POOL["data"]
+    if kind == "prefill":
+        _oracle_prefill_rows(PREFILL_WL[name], data, arg)
+    elif kind == "chunk":
+        _oracle_chunk(CHUNK_WL[name], data, arg)
+    else:
+        wl = DECODE_WL[name]
+        _oracle_decode(wl, data["dq"], data["cache"], arg, data["firsts"])
+    return len(arg)
+
+
+def _shared(x):
+    """Tensors (also inside dicts and lists) moved to shared memory for the workers."""
+    if torch.is_tensor(x):
+        return x.share_memory_()
+    if isinstance(x, dict):
+        return {k: _shared(v) for k, v in x.items()}
+    if isinstance(x, (list, tuple)):
+        return type(x)(_shared(v) for v in x)
+    return x
+
+
+def _pool_size(per_worker_bytes: float) -> int:
+    n = os.cpu_count() or 1
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+        n = min(n, int(avail * 0.6 // max(per_worker_bytes, 1.0)))
+    except Exception:
+        pass
+    return max(1, n)
+
+
+class OraclePool:
+    """A spawn-context process pool holding one workload's inputs."""
+
+    def __init__(self, name):
+        import concurrent.futures as cf
+        import torch.multiprocessing as tmp
+        if name in CHUNK_WL:
+            wl = CHUNK_WL[name]
+            kind, data = "chunk", W.chunk_inputs(wl)
+            per = 8.0 * 4 * sum(t.numel() for t in data.values() if torch.is_tensor(t))
+        elif name in PREFILL_WL:
+            wl = PREFILL_WL[name]
+            kind, data = "prefill", W.prefill_inputs(wl)
+            per = 8.0 * 2 * sum(t.numel() for t in data.values() if torch.is_tensor(t))
+        else:
+            wl = DECODE_WL[name]
+            dq = W.decode_inputs(wl)
+            lens = dq["seq_lens"].numpy()
+            L = wl.layer
+            ks, vs, firsts = [], [], []
+            for b in range(wl.batch):
+                n = int(lens[b])
+                lo = 0 if L.window == 0 else max(0, n - L.window)
+                rows = W.decode_cache_rows(wl, b, n - lo, lo)
+                ks.append(rows["k"])
+                vs.append(rows["v"])
+                firsts.append(lo)
+            cache = _oracle_cache(wl, ks, vs, firsts)
+            kind, data = "decode", dict(dq=dq, cache=cache, firsts=firsts)
+            per = 8.0 * 4 * max(int(n) for n in lens) * L.num_kv_heads * L.head_dim
+        self.kind, self.name, self.wl, self.data = kind, name, wl, data
+        self.workers = _pool_size(per + 256e6)
+        self.ex = cf.ProcessPoolExecutor(self.workers, mp_context=tmp.get_context("spawn"), initializer=_pool_init,
+                                         initargs=(kind, name, _shared(data)))
+        # start every worker (initializer, imports, first-call costs) before any timing
+        first = np.array([0]) if kind != "decode" else [0]
+        list(self.ex.map(_pool_task, [first] * self.workers))
+
+    def run(self, tasks):
+        """Wall seconds to run every task, spread over the pool."""
         t0 = time.perf_counter()
-        _oracle_prefill_rows(wl, d, pilot)
-        per_row = (time.perf_counter() - t0) / len(pilot)
-        n = int(max(8, min(S, budget_s / max(per_row, 1e-6))))
-        rows = np.unique(np.linspace(0, S - 1, n).astype(np.int64))
-        # the pilot's per-row cost carries the per-call key transform, so the strided
-        # sample can finish well inside the budget: repeat it until about two thirds of
-        # the budget is spent (at most 16 passes)
-        dt, reps = 0.0, 0
-        while reps < 16 and (reps == 0 or dt < budget_s * 2 / 3):
-            t0 = time.perf_counter()
-            _oracle_prefill_rows(wl, d, rows)
-            dt += time.perf_counter() - t0
-            reps += 1
-        L = wl.layer
-        work = rows_flops(wl, d, rows) * reps
-        return {"value": round(work / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
-                "kind": "oracle",
-                "sample": f"{len(rows)} evenly spaced query rows of {S}, all {wl.batch} sequences and "
-                          f"{L.num_heads} heads, {reps} pass(es) ({dt:.1f} s, float64 numpy)"}
-    wl = DECODE_WL[name]
-    dq = W.decode_inputs(wl)
-    lens = dq["seq_lens"].numpy()
-    L = wl.layer
-    done, t0, ks, vs, firsts = [], time.perf_counter(), [], [], []
-    for b in range(wl.batch):
-        n = int(lens[b])
-        lo = 0 if L.window == 0 else max(0, n - L.window)
-        rows = W.decode_cache_rows(wl, b, n - lo, lo)
-        ks.append(rows["k"])
-        vs.append(rows["v"])
-        firsts.append(lo)
-    cache = _oracle_cache(wl, ks, vs, firsts)
-    t0 = time.perf_counter()
-    for b in range(wl.batch):
-        _oracle_decode(wl, dq, cache, [b], firsts)
-        done.append(b)
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    work = decode_bytes(L, lens[done], wl.kv_int8)
-    return {"value": round(work / dt / 1e9, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{len(done)} of {wl.batch} batch rows ({dt:.1f} s, float64 numpy)"}
+        list(self.ex.map(_pool_task, tasks))
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.ex.shutdown()
+
+
+def _row_tasks(rows, nchunks):
+    """Interleaved row blocks, so that causal costs spread evenly over the blocks."""
+    rows = np.asarray(rows)
+    return [rows[i::nchunks] for i in range(min(nchunks, len(rows))) if len(rows[i::nchunks])]
+
+
+def cpu_baseline(name, budget_s=15.0):
+    """The oracle timed on a strided sample of query rows (prefill, chunk) or on the batch rows
+    (decode) of the workload, over a process pool on the host cores."""
+    pool = OraclePool(name)
+    try:
+        P = pool.workers
+        if pool.kind in ("prefill", "chunk"):
+            wl = pool.wl
+            n_all = wl.seq if pool.kind == "prefill" else wl.chunk
+            # pilot: one block of rows on one worker sizes the sample to about the budget
+            pilot = np.unique(np.linspace(0, n_all - 1, min(n_all, 8)).astype(np.int64))
+            t_pilot = pool.run([pilot])
+            per_row = t_pilot / len(pilot)
+            n = int(max(P, min(n_all, budget_s * P / max(per_row, 1e-9))))
+            rows = np.unique(np.linspace(0, n_all - 1, n).astype(np.int64))
+            dt = pool.run(_row_tasks(rows, 2 * P))
+            if pool.kind == "prefill":
+                work = rows_flops(wl, pool.data, rows)
+                what = f"query rows of {n_all}, all {wl.batch} sequences and {wl.layer.num_heads} heads"
+            else:
+                work = chunk_flops(wl, rows)
+                what = f"chunk rows of {n_all}, all {wl.batch} sequences and {wl.layer.num_heads} heads"
+            return {"value": round(work / dt / 1e12, 6), "unit": "TFLOP/s", "cores": P, "kind": "oracle",
+                    "sample": f"{len(rows)} evenly spaced {what}, in {min(2 * P, len(rows))} blocks over {P} "
+                              f"worker processes, one BLAS thread each ({dt:.1f} s wall, float64 numpy)"}
+        wl = pool.wl
+        lens = pool.data["dq"]["seq_lens"].numpy()
+        dt = pool.run([[b] for b in range(wl.batch)])
+        work = decode_bytes(wl.layer, lens, wl.kv_int8)
+        return {"value": round(work / dt / 1e9, 4), "unit": "GB/s", "cores": P, "kind": "oracle",
+                "sample": f"all {wl.batch} batch rows, one per task over {P} worker processes, one BLAS thread "
+                          f"each ({dt:.1f} s wall, float64 numpy)"}
+    finally:
+        pool.close()
 
 
 def run_reference(args, world, rank):
-    """The oracle as the reference arm: each step is a bounded sample of the same workload."""
+    """The oracle as the reference arm: each step is a bounded sample of the same workload,
+    spread over a process pool on the host cores."""
     if rank != 0:
         return None
-    import oracle as O  # noqa: F401
     name = args.workload
     budget = float(os.environ.get("GATTN_REF_BUDGET_S", "120"))
     n_steps = args.steps + args.warmup
-    if name in CHUNK_WL:
-        wl = CHUNK_WL[name]
-        d = W.chunk_inputs(wl)
-        t0 = time.perf_counter()
-        _oracle_chunk(wl, d, np.array([wl.chunk - 1]))
-        per_row = time.perf_counter() - t0
-        rows_per_step = int(max(1, min(wl.chunk, budget / n_steps / max(per_row, 1e-6))))
+    pool = OraclePool(name)
+    try:
+        P = pool.workers
+        wl = pool.wl
         rng = np.random.default_rng(0)
         work, dt = 0.0, 0.0
-        for i in range(n_steps):
-            rows = np.sort(rng.choice(wl.chunk, size=rows_per_step, replace=False))
-            t0 = time.perf_counter()
-            _oracle_chunk(wl, d, rows)
-            el = time.perf_counter() - t0
-            if i >= args.warmup:
-                dt += el
-                work += chunk_flops(wl, rows)
-        value, unit = work / dt / 1e12, "TFLOP/s"
-        sample = f"{rows_per_step} random chunk rows of {wl.chunk} per step, all sequences and heads"
-        metric = "attention prefill TFLOP/s (effective FLOPs)"
-    elif name in PREFILL_WL:
-        wl = PREFILL_WL[name]
-        d = W.prefill_inputs(wl)
-        S, L = wl.seq, wl.layer
-        t0 = time.perf_counter()
-        _oracle_prefill_rows(wl, d, np.array([S - 1]))
-        per_row = time.perf_counter() - t0
-        rows_per_step = int(max(1, min(S, budget / n_steps / max(per_row, 1e-6))))
-        rng = np.random.default_rng(0)
-        work, dt = 0.0, 0.0
-        for i in range(n_steps):
-            rows = np.sort(rng.choice(S, size=rows_per_step, replace=False))
-            t0 = time.perf_counter()
-            _oracle_prefill_rows(wl, d, rows)
-            el = time.perf_counter() - t0
-            if i >= args.warmup:
-                dt += el
-                work += rows_flops(wl, d, rows)
-        value, unit = work / dt / 1e12, "TFLOP/s"
-        sample = f"{rows_per_step} random query rows of {S} per step, all sequences and heads"
-        metric = "attention prefill TFLOP/s (effective FLOPs)"
-    else:
-        wl = DECODE_WL[name]
-        dq = W.decode_inputs(wl)
-        lens = dq["seq_lens"].numpy()
-        L = wl.layer
-        work, dt = 0.0, 0.0
-        for i in range(n_steps):
-            b = i % wl.batch
-            n = int(lens[b])
-            lo = 0 if L.window == 0 else max(0, n - L.window)
-            rows = W.decode_cache_rows(wl, b, n - lo, lo)
-            ks = [rows["k"] if j == b else None for j in range(wl.batch)]
-            vs = [rows["v"] if j == b else None for j in range(wl.batch)]
-            fr = [lo if j == b else 0 for j in range(wl.batch)]
-            cache = _oracle_cache(wl, ks, vs, fr)
-            t0 = time.perf_counter()
-            _oracle_decode(wl, dq, cache, [b], fr)
-            el = time.perf_counter() - t0
-            if i >= args.warmup:
-                dt += el
-                work += decode_bytes(L, lens[b:b + 1], wl.kv_int8)
-        value, unit = work / dt / 1e9, "GB/s"
-        sample = "one batch row per step, cycling over the batch"
-        metric = "decode KV GB/s (algorithmic bytes)"
-    cores = blas_threads()
+        if pool.kind in ("prefill", "chunk"):
+            n_all = wl.seq if pool.kind == "prefill" else wl.chunk
+            per_row = pool.run([np.array([n_all - 1])])
+            rows_per_step = int(max(1, min(n_all, budget * P / n_steps / max(per_row, 1e-9))))
+            for i in range(n_steps):
+                rows = np.sort(rng.choice(n_all, size=rows_per_step, replace=False))
+                el = pool.run(_row_tasks(rows, 2 * P))
+                if i >= args.warmup:
+                    dt += el
+                    work += rows_flops(wl, pool.data, rows) if pool.kind == "prefill" else chunk_flops(wl, rows)
+            value, unit = work / dt / 1e12, "TFLOP/s"
+            sample = (f"{rows_per_step} random {'query' if pool.kind == 'prefill' else 'chunk'} rows of {n_all} per "
+                      f"step, all sequences and heads, over {P} worker processes (one BLAS thread each)")
+            metric = "attention prefill TFLOP/s (effective FLOPs)"
+        else:
+            lens = pool.data["dq"]["seq_lens"].numpy()
+            per_step = min(wl.batch, P)
+            for i in range(n_steps):
+                bs = [int(b) for b in rng.choice(wl.batch, size=per_step, replace=False)]
+                el = pool.run([[b] for b in bs])
+                if i >= args.warmup:
+                    dt += el
+                    work += decode_bytes(wl.layer, lens[bs], wl.kv_int8)
+            value, unit = work / dt / 1e9, "GB/s"
+            sample = f"{per_step} random batch rows per step, one per task over {P} worker processes"
+            metric = "decode KV GB/s (algorithmic bytes)"
+    finally:
+        pool.close()
     return {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / max(args.steps, 1) * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": name},
-            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": P, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

@@ -46,7 +46,7 @@ namespace {
 constexpr int kSW = 8;                  // compute warps
 constexpr int kTileBytes = 32768;       // bf16 cache bytes per tile (keys; values as many); int8: half
 constexpr int kTabBytes = 8192;         // RoPE table rows of a tile, staged when they fit
-constexpr int kPlanSMs = 148;           // work-item target for the split plan (B200 SM count)
+
 constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n >> 1); }
@@ -702,6 +702,20 @@ __global__ void __launch_bounds__(kSW * 32, 1) decode_simt_kernel(const __grid_c
 
 namespace {
 
+// SM count of the current device, queried once per device (148 if the query fails).
+int device_sm_count() {
+  constexpr int kMaxDev = 64;
+  static int sms[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
 template <int D, int G, bool KEQV, bool Q8>
 cudaError_t run_decode_simt(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
   using C = SimtShape<D, G, KEQV, Q8>;
@@ -746,7 +760,8 @@ void decode_simt_plan(const LayerArgs& la, int B, int max_len, int max_split, in
   const int SUB = kSW / la.Hkv;
   const int TP = kTileBytes / (2 * la.D) / la.Hkv;
   const int span = la.window > 0 ? (la.window < max_len ? la.window : max_len) : max_len;
-  int nch = (16 * kPlanSMs + (B > 0 ? B : 1) - 1) / (B > 0 ? B : 1);
+  const int sms = device_sm_count();
+  int nch = (16 * sms + (B > 0 ? B : 1) - 1) / (B > 0 ? B : 1);
   const int tiles = (span + TP - 1) / TP;
   if (nch > tiles) nch = tiles;
   if (nch > 64) nch = 64;

@@ -9,6 +9,7 @@
 // second kernel merges them with the log-sum-exp rule.
 #include <cuda_bf16.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "gattn_internal.h"
@@ -474,9 +475,19 @@ static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, c
   const size_t smem = sizeof(float) * (static_cast<size_t>(la.G) * D + 2 * kDecodeWarps * HPW +
                                        static_cast<size_t>(kDecodeWarps) * HPW * D);
   auto kern = decode_split_kernel<NCH, HPW>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  // the shared-memory opt-in is per device and per size: set it when a call
+  // needs more than this device was last given (never on every call)
+  constexpr int kMaxDev = 64;
+  static size_t attr_smem[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (smem > attr_smem[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_smem[dev] = smem;
+  }
   dim3 grid(da.nsplit, la.Hkv, da.B);
   kern<<<grid, kDecodeWarps * 32, smem, s>>>(da, la);
   return cudaGetLastError();
@@ -585,10 +596,18 @@ extern "C" int gattn_decode_noalloc(const gattn_bf16* q, const gattn_bf16* k_cac
   const size_t fit = usable / per_split;
   const int max_split = fit > (1u << 30) ? (1 << 30) : static_cast<int>(fit);
   if (max_split >= 1) decode_plan(la, batch, max_len, &da.nsplit, &da.chunk, max_split);
-  if (max_split < 1 || da.nsplit > max_split)
-    return report_error(GATTN_ERR_UNSUPPORTED,
-                        "batch * num_heads * (head_dim + 2) * 4 bytes exceed the 16 MiB scratch "
-                        "of gattn_decode_noalloc; use gattn_decode with a workspace");
+  if (max_split < 1 || da.nsplit > max_split) {
+    // the layer's smallest plan still needs more split slots than fit: one
+    // slot per chunk, and on the CUDA-core kernel's layers a chunk takes one
+    // slot per warp-row group (8 / num_kv_heads of them)
+    char msg[256];
+    std::snprintf(msg, sizeof(msg),
+                  "the smallest split plan of this layer needs %d slots of batch * num_heads * (head_dim + 2) * "
+                  "4 = %zu bytes, more than the 16 MiB scratch of gattn_decode_noalloc holds (%d); use "
+                  "gattn_decode with a workspace",
+                  max_split < 1 ? 1 : da.nsplit, per_split, max_split < 0 ? 0 : max_split);
+    return report_error(GATTN_ERR_UNSUPPORTED, msg);
+  }
   void* base = nullptr;
   cudaError_t e = noalloc_scratch_address(&base);
   if (e != cudaSuccess) return report_error(GATTN_ERR_CUDA, "cudaGetSymbolAddress of the decode scratch failed");

@@ -275,12 +275,18 @@ int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k
  * and may return wrong results; order them on one stream.  Nothing in the
  * array needs to start at zero (every partial is written before it is read),
  * and it keeps the last call's partials.
- * If batch * num_heads * (head_dim + 2) * 4 bytes exceed the array, it returns
- * GATTN_ERR_UNSUPPORTED and enqueues nothing; otherwise it uses fewer, longer
- * splits when the normal split count would not fit.  There is no status word,
- * so kernel-side range errors (a seq_lens entry outside [1, max_len], a
- * position past the RoPE table) are not reported: such rows are written as
- * zeros / clamped exactly as gattn_decode does. */
+ * A split slot takes batch * num_heads * (head_dim + 2) * 4 bytes.  When the
+ * normal split count would not fit, it uses fewer, longer splits; if even the
+ * layer's smallest plan does not fit (one slot per chunk, and, on layers with
+ * 1, 2 or 4 query heads per kv head, which run on the CUDA-core kernel,
+ * 8 / num_kv_heads slots per chunk), it returns GATTN_ERR_UNSUPPORTED and
+ * enqueues nothing.  There is no status word, so nothing device-side is
+ * reported: kernel-side range errors (a seq_lens entry outside [1, max_len],
+ * a position past the RoPE table) are handled as gattn_decode handles them
+ * (rows written as zeros / positions clamped), and if a kernel's bounded wait
+ * runs out (the 2 s default of gattn_set_wait_timeout_us), the key chunk that
+ * split was reading is left out of the merge: the call returns a finite but
+ * wrong result for that row without any error. */
 int gattn_decode_noalloc(const gattn_bf16* q, const gattn_bf16* k_cache,
                          const gattn_bf16* v_cache_or_null, const int32_t* seq_lens, gattn_bf16* out,
                          int32_t batch, int32_t max_len, const gattn_cfg* cfg, gattn_stream stream);
@@ -333,6 +339,12 @@ void gattn_set_profile_events(void* start_event, void* stop_event);
  * P^T complete (seen by the P V issuer), [296+j] angles advanced, and
  * per-warp completion of the key prologue ([320/344/368+j], warps 5-7) and
  * of the softmax ([392/416/440+j], warps 1-3).
+ * Whole prompts of head_dim-512 layers with an even number of query heads per
+ * kv head run on SM pairs: there CTA i of the first bytes/4096 writes [0]
+ * start, [1] SM id, [2] its rank in the pair, [3] items it takes, [4] key
+ * tiles of its first item, and per key tile j < 120 of that item [8+j] S(j)
+ * seen by the softmax, [128+j] P(j) written, and (first CTA of the pair)
+ * [248+j] Q K^T(j) issued, [368+j] P V(j) issued.
  * A debugging aid; NULL turns it off. */
 void gattn_set_trace_buffer(void* device_buffer, size_t bytes);
 
