@@ -195,6 +195,25 @@ const char* gattn_status_string(int s) {
 
 const char* gattn_last_error(void) { return g_last_error; }
 
+int gattn_cp_blocks(int32_t seq_len, int32_t world, int32_t rank, int32_t* starts, int32_t* lens) {
+  g_last_error[0] = 0;
+  if (!starts || !lens) return fail(GATTN_ERR_INVALID_ARG, "starts and lens must not be NULL");
+  if (world < 1) return fail(GATTN_ERR_INVALID_ARG, "world must be >= 1");
+  if (rank < 0 || rank >= world) return fail(GATTN_ERR_INVALID_ARG, "rank must be in [0, world)");
+  if (seq_len < 0) return fail(GATTN_ERR_INVALID_ARG, "seq_len must be >= 0");
+  const int64_t nb = 2 * static_cast<int64_t>(world);
+  const int64_t base = seq_len / nb, extra = seq_len % nb;
+  // block i: base tokens, one more for the first `extra` blocks
+  auto start_of = [&](int64_t i) { return i * base + (i < extra ? i : extra); };
+  auto len_of = [&](int64_t i) { return base + (i < extra ? 1 : 0); };
+  const int64_t b0 = rank, b1 = nb - 1 - rank;
+  starts[0] = static_cast<int32_t>(start_of(b0));
+  lens[0] = static_cast<int32_t>(len_of(b0));
+  starts[1] = static_cast<int32_t>(start_of(b1));
+  lens[1] = static_cast<int32_t>(len_of(b1));
+  return GATTN_OK;
+}
+
 void gattn_set_wait_timeout_us(uint32_t timeout_us) {
   g_timeout_ns = (timeout_us ? static_cast<uint64_t>(timeout_us) : 2000000ull) * 1000ull;
 }

@@ -29,7 +29,7 @@ EXPORTS = ("gattn_version", "gattn_status_string", "gattn_last_error", "gattn_ro
            "gattn_selftest_wait_timeout", "gattn_set_wait_timeout_us", "gattn_set_profile_events",
            "gattn_set_trace_buffer", "gattn_decode_noalloc", "gattn_prefill_padded", "gattn_kv_quantize",
            "gattn_decode_int8", "gattn_prefill_chunk_workspace_size", "gattn_prefill_chunk", "gattn_kv_append",
-           "gattn_kv_append_layer")
+           "gattn_kv_append_layer", "gattn_cp_blocks")
 
 
 class GattnError(RuntimeError):
@@ -116,6 +116,8 @@ def lib() -> ctypes.CDLL:
         L.gattn_kv_quantize.argtypes = [vp, vp, vp, ctypes.c_int64, i32, vp]
         L.gattn_decode_int8.restype = ctypes.c_int
         L.gattn_decode_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz, vp]
+        L.gattn_cp_blocks.restype = ctypes.c_int
+        L.gattn_cp_blocks.argtypes = [i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         L.gattn_prefill_padded.restype = ctypes.c_int
         L.gattn_prefill_padded.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(GattnCfg), vp, sz,
                                            vp]
@@ -406,3 +408,12 @@ def set_trace_buffer(buf: Optional[torch.Tensor] = None):
 
 def version() -> str:
     return lib().gattn_version().decode()
+
+
+def cp_blocks(seq_len: int, world: int, rank: int):
+    """gattn_cp_blocks: rank's two token blocks [(start, len), (start, len)] of a prompt of
+    seq_len tokens split over `world` ranks (zig-zag: blocks rank and 2*world-1-rank of 2*world)."""
+    starts = (ctypes.c_int32 * 2)()
+    lens = (ctypes.c_int32 * 2)()
+    _raise_if(lib().gattn_cp_blocks(seq_len, world, rank, starts, lens), "gattn_cp_blocks")
+    return [(int(starts[0]), int(lens[0])), (int(starts[1]), int(lens[1]))]

@@ -206,6 +206,25 @@ int gattn_kv_append_layer(const gattn_cfg* cfg, const gattn_bf16* k_new, const g
                           int32_t batch, int32_t n_new, int32_t max_len, void* status_or_null,
                           gattn_stream stream);
 
+/* ---- context parallelism: one long prompt over several GPUs --------------------
+ * The model cards give Gemma 4 a 256K context window (KerasFormers "Gemma 4"),
+ * and the Atlas "Gemma 4" summary trains with the data sharded by sequence as
+ * well as by batch and replica; one prompt that long is split over the GPUs of
+ * a node by query rows.  gattn_cp_blocks is the split: the prompt's seq_len
+ * tokens are cut into 2 * world contiguous blocks as evenly as possible (the
+ * first seq_len mod (2 * world) blocks one token longer), and rank r owns
+ * blocks r and 2 * world - 1 - r, so that every rank's causal work (the
+ * visible pairs of its query rows) is the same to within one block's rows.
+ * Each rank then gathers every rank's key (and value) rows of its blocks (one
+ * all-gather over the node's links; with k_eq_v one tensor), and runs each of
+ * its two blocks as a chunk (gattn_prefill_chunk with the gathered keys as the
+ * cache, prefix_lens = the block's first token, no append): a block's rows
+ * see exactly the keys a whole-prompt prefill gives them.
+ * Writes starts[0..1] and lens[0..1] (host int32): rank's two blocks in token
+ * order.  Host only; returns GATTN_OK, or GATTN_ERR_INVALID_ARG for world < 1,
+ * rank outside [0, world), seq_len < 0 or NULL pointers. */
+int gattn_cp_blocks(int32_t seq_len, int32_t world, int32_t rank, int32_t* starts, int32_t* lens);
+
 /* ---- decode ----------------------------------------------------------------
  * One decode step: query b (at position seq_lens[b]-1) against cache rows
  * [0, seq_lens[b]) of its own cache.  Caches hold RAW keys/values (before
