@@ -43,17 +43,20 @@ using bf16 = __nv_bfloat16;
 
 namespace {
 
+template <int D_>
 struct PairShape {
-  static constexpr int D = 512;
+  static constexpr int D = D_;
   static constexpr int BM = 128;                   // query rows per CTA
   static constexpr int BN = 128;                   // keys per tile (64 per CTA for Q K^T)
   static constexpr int DV = 256;                   // value dims per item (128 per CTA for P V)
+  static_assert(D == 256 || D == 512, "head_dim 256 or 512");
   static constexpr int QBOX = BM * 128;            // 64 dims x 128 rows, 128-byte swizzle
   static constexpr int Q_BYTES = (D / 64) * QBOX;  // 128 KB
   static constexpr int KBOX = 8192;                // key box: 64 dims x this CTA's 64 keys
   static constexpr int VBOX = 16384;               // value box: 64 dims x 128 keys
   static constexpr int UNIT = 4 * KBOX;            // one barrier phase: 32 KB per CTA
-  static constexpr int NUNIT = 3;                  // ring of 96 KB
+  static constexpr int DVS = D / 256;              // work items per query tile and head pair (value halves)
+  static constexpr int NUNIT = (232448 - Q_BYTES - 1536) / UNIT;  // ring: 3 units at D 512, 5 at D 256
   static constexpr int KUNITS = D / 256;           // units of a key tile (256 dims each)
   static constexpr int VUNITS = 1;                 // units of a value tile (this CTA's 128 dims)
   static_assert(2 * VBOX == UNIT, "a value tile fills one unit");
@@ -88,10 +91,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace
 
-template <bool CAP>
+template <int D, bool CAP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     prefill_pair_kernel(const __grid_constant__ PairParams P) {
-  using C = PairShape;
+  using C = PairShape<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   // identical kernels, so the aligned offsets agree between the two CTAs
@@ -114,7 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const uint32_t rank = cluster_ctarank();
   const LayerArgs& la = P.la;
   const int H = la.H, S = P.S;
-  const int per_qt = P.B * la.Hkv * P.npairs * 2;
+  const int per_qt = P.B * la.Hkv * P.npairs * C::DVS;
   const int nitems = P.nqt * per_qt;
   struct Item {
     int qt, dvs, h, b, kvh, q0, dv_lo, k_first, ntiles, rot;
@@ -123,8 +126,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     Item w;
     w.qt = P.nqt - 1 - it / per_qt;
     int idx = it % per_qt;
-    w.dvs = idx & 1;
-    idx >>= 1;
+    w.dvs = idx % C::DVS;
+    idx /= C::DVS;
     const int pg = idx % P.npairs;
     idx /= P.npairs;
     w.kvh = idx % la.Hkv;
@@ -137,8 +140,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     w.k_first = (kv_lo / BN) * BN;
     w.ntiles = (kv_hi - w.k_first + BN - 1) / BN;
     // items reading one sequence at once start at different key tiles, so
-    // they do not all read the same L2 lines together (the order is free)
-    w.rot = w.ntiles > 1 ? (pg * 7 + w.kvh * 3 + w.b * 5 + w.qt + w.dvs * 11) % w.ntiles : 0;
+    // they do not all read the same L2 lines together (the order is free; it
+    // follows the pair's first head, so a layout of the same heads over more
+    // kv heads visits the same tiles in the same order)
+    w.rot = w.ntiles > 1 ? ((w.h - static_cast<int>(rank)) * 7 + w.b * 5 + w.qt + w.dvs * 11) % w.ntiles : 0;
     return w;
   };
   auto tile_key = [&](const Item& w, int j) { return w.k_first + ((j + w.rot) % w.ntiles) * BN; };
@@ -514,11 +519,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
+// head_dim 512 only: at head_dim 256 the single-SM kernel holds both tiles'
+// operands within shared memory's bandwidth, and the pair measured slower
+// (Gemma-1 MQA prefill 738 against 920 TFLOP/s, Gemma-3 global 1087 against 1310)
 bool prefill_pair_supported(const LayerArgs& la) { return la.D == 512 && la.G % 2 == 0; }
 
-cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
-  using C = PairShape;
-  if (!prefill_pair_supported(la) || pa.seq_range || pa.q_off) return cudaErrorInvalidValue;
+template <int D>
+static cudaError_t run_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+  using C = PairShape<D>;
   PairParams P;
   if (!encode_tmap_bshd(&P.tm_q, pa.q, pa.B, pa.S, la.H, C::D, C::BM) ||
       !encode_tmap_bshd(&P.tm_k, pa.kt, pa.B, pa.S, la.Hkv, C::D, C::BN / 2) ||
@@ -535,13 +543,13 @@ cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cuda
   P.trace = pa.trace;
   P.trace_ctas = static_cast<int>(pa.trace_bytes / (512 * sizeof(unsigned long long)));
   const bool cap = la.softcap > 0.f;
-  auto kern = cap ? prefill_pair_kernel<true> : prefill_pair_kernel<false>;
+  auto kern = cap ? prefill_pair_kernel<D, true> : prefill_pair_kernel<D, false>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   // per device: the shared-memory opt-in and how many pairs can be resident
   constexpr int kMaxDev = 64;
-  static int max_clusters[kMaxDev][2] = {};
+  static int max_clusters[kMaxDev][2] = {};  // per instance (D fixed here), per softcap
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
   int& mc = max_clusters[dev][cap ? 1 : 0];
   if (mc == 0) {
@@ -557,10 +565,15 @@ cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cuda
     if (n < 1) return cudaErrorInvalidConfiguration;
     mc = n;
   }
-  const long long items = static_cast<long long>(P.nqt) * pa.B * la.Hkv * P.npairs * 2;
+  const long long items = static_cast<long long>(P.nqt) * pa.B * la.Hkv * P.npairs * C::DVS;
   if (items > (1LL << 31) - 1) return cudaErrorInvalidValue;
   const long long nc = items < mc ? items : mc;
   return launch_pdl(kern, dim3(static_cast<unsigned>(2 * nc)), dim3(192), C::SMEM, s, P);
+}
+
+cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
+  if (!prefill_pair_supported(la) || pa.seq_range || pa.q_off) return cudaErrorInvalidValue;
+  return run_pair<512>(pa, la, s);
 }
 
 }  // namespace gattn
