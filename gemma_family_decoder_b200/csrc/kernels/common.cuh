@@ -396,6 +396,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
 // Expect `bytes` of asynchronous copies on an mbarrier of any CTA of the
 // cluster and arrive on it; relaxed: the arriving thread orders no data of its
 // own (the copies' bytes complete the phase), so no cluster-wide fence.
+// Arrive on an mbarrier of any CTA of the cluster with CTA-scope release: for
+// signals whose data is in tensor memory (ordered by the tcgen05 fences around
+// the thread synchronisation), not in shared or global memory.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_cluster_addr, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
                    bar_cluster_addr),

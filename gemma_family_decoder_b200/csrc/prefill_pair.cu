@@ -27,6 +27,7 @@
 //              CTA's barrier.
 //   warp 5     (first CTA only) issues the pair MMAs and their commits, which
 //              arrive on the matching barriers of both CTAs.
+//   warp 6     a second TMA producer (alternate ring units).
 // Clusters are persistent and take items heaviest first in zig-zag rounds.
 //
 // Layer definition: KerasFormers "Gemma 4" (What changed: global layers with
@@ -92,7 +93,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace
 
 template <int D, bool CAP>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     prefill_pair_kernel(const __grid_constant__ PairParams P) {
   using C = PairShape<D>;
   constexpr int BN = C::BN;
@@ -171,7 +172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if ((warp == 4 || warp == 6) && lane == 0) {
     tma_prefetch_desc(&P.tm_q);
     tma_prefetch_desc(&P.tm_k);
     tma_prefetch_desc(&P.tm_v);
@@ -318,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         // the warp's tensor-memory stores are complete (wait::st is warp-wide):
         // one cluster-scope arrival per warp instead of one fence per thread
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(p_full_l[T & 1]);
+        if (lane == 0) mbar_arrive_remote(p_full_l[T & 1]);
         if (t == 0 && I == 0 && j < 120) mark(128 + j);
       }
       ok = ok && __all_sync(0xffffffffu, mbar_wait(o_final, I & 1, tmo, P.status, abort_flag));
@@ -348,26 +349,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(o_empty_l);
+      if (lane == 0) mbar_arrive_remote(o_empty_l);
       T0 += w.ntiles;
       ++I;
     }
-  } else if (warp == 4) {
-    // ------------------------------------------------------------------ producer
+  } else if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------------ producers
     // Units are issued in the order the MMAs consume them: the key units of
     // tile 0, this CTA's Q tile, then per tile j the key units of j and the
     // value unit of j - 1.  A key unit holds this CTA's 64 keys of the tile at
     // 256 dims (four boxes); a value unit all 128 keys at this CTA's 128 value
-    // dims (two boxes).
+    // dims (two boxes).  Two threads in two warps issue alternate units (and
+    // the first the Q tiles): one thread's copy stream is limited by a fixed
+    // cost per barrier phase, which a second issuing thread halves.
     if (lane == 0) {
-      int n = 0;  // units issued
+      const int pid = warp == 4 ? 0 : 1;
+      int n = 0;  // units of the sequence so far (either thread's)
       auto acquire = [&](int& u) -> bool {
         u = n % C::NUNIT;
         return mbar_wait(&empty[u], ((n / C::NUNIT) & 1) ^ 1, tmo, P.status, abort_flag);
       };
       auto load_k = [&](const Item& w, int j) -> bool {
         const int key = tile_key(w, j) + static_cast<int>(rank) * (BN / 2);
-        for (int ku = 0; ku < C::KUNITS; ++ku) {
+        for (int ku = 0; ku < C::KUNITS; ++ku, ++n) {
+          if ((n & 1) != pid) continue;
           int u;
           if (!acquire(u)) return false;
           const uint32_t lb = leader(&full[u]);
@@ -376,13 +381,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             tma_load_4d_pair(dst + c * C::KBOX, &P.tm_k, lb, ku * 256 + c * 64, w.kvh, key, w.b);
-          ++n;
         }
         return true;
       };
       auto load_v = [&](const Item& w, int j) -> bool {
         const int dv = w.dv_lo + static_cast<int>(rank) * (C::DV / 2);
-        for (int vu = 0; vu < C::VUNITS; ++vu) {
+        for (int vu = 0; vu < C::VUNITS; ++vu, ++n) {
+          if ((n & 1) != pid) continue;
           int u;
           if (!acquire(u)) return false;
           const uint32_t lb = leader(&full[u]);
@@ -391,7 +396,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const int key = tile_key(w, j);
           tma_load_4d_pair(dst, &P.tm_v, lb, dv, w.kvh, key, w.b);
           tma_load_4d_pair(dst + C::VBOX, &P.tm_v, lb, dv + 64, w.kvh, key, w.b);
-          ++n;
         }
         return true;
       };
@@ -404,13 +408,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const Item w = item_of(it);
         ok = load_k(w, 0);
         if (!ok) break;
-        ok = mbar_wait(q_empty, (I & 1) ^ 1, tmo, P.status, abort_flag);
-        if (!ok) break;
-        mbar_arrive_expect_tx_cluster(q_full_l, C::Q_BYTES);
+        if (pid == 0) {
+          ok = mbar_wait(q_empty, (I & 1) ^ 1, tmo, P.status, abort_flag);
+          if (!ok) break;
+          mbar_arrive_expect_tx_cluster(q_full_l, C::Q_BYTES);
 #pragma unroll 1
-        for (int c = 0; c < C::D / 64; ++c)
-          tma_load_4d_pair(smem + C::OFF_Q + c * C::QBOX, &P.tm_q, q_full_l, c * 64, w.h, w.q0, w.b);
-        lq = I;
+          for (int c = 0; c < C::D / 64; ++c)
+            tma_load_4d_pair(smem + C::OFF_Q + c * C::QBOX, &P.tm_q, q_full_l, c * 64, w.h, w.q0, w.b);
+          lq = I;
+        }
         for (int j = 1; j < w.ntiles && ok; ++j) {
           ok = load_k(w, j);
           if (ok) ok = load_v(w, j - 1);
@@ -421,7 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       // every copy issued lands before the CTA can exit: the MMAs that read
       // the last NUNIT units (and the last Q tile) completed, so did their copies
       for (int k = n - C::NUNIT > 0 ? n - C::NUNIT : 0; k < n; ++k)
-        mbar_wait(&empty[k % C::NUNIT], (k / C::NUNIT) & 1, tmo, P.status, nullptr);
+        if ((k & 1) == pid) mbar_wait(&empty[k % C::NUNIT], (k / C::NUNIT) & 1, tmo, P.status, nullptr);
       if (lq >= 0) mbar_wait(q_empty, lq & 1, tmo, P.status, nullptr);
     }
   } else if (rank == 0) {
@@ -557,7 +563,7 @@ static cudaError_t run_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStre
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t qc = {};
     qc.gridDim = dim3(2);
-    qc.blockDim = dim3(192);
+    qc.blockDim = dim3(224);
     qc.dynamicSmemBytes = C::SMEM;
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, kern, &qc);
@@ -568,7 +574,7 @@ static cudaError_t run_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStre
   const long long items = static_cast<long long>(P.nqt) * pa.B * la.Hkv * P.npairs * C::DVS;
   if (items > (1LL << 31) - 1) return cudaErrorInvalidValue;
   const long long nc = items < mc ? items : mc;
-  return launch_pdl(kern, dim3(static_cast<unsigned>(2 * nc)), dim3(192), C::SMEM, s, P);
+  return launch_pdl(kern, dim3(static_cast<unsigned>(2 * nc)), dim3(224), C::SMEM, s, P);
 }
 
 cudaError_t launch_prefill_pair(const PrefillArgs& pa, const LayerArgs& la, cudaStream_t s) {
