@@ -348,16 +348,6 @@ void gattn_set_profile_events(void* start_event, void* stop_event);
  * [3] Q ready, [4] epilogue start, [5] end, [6] first key box landed, and per
  * key tile j < 120: [8+j] S(j) seen by the softmax, [128+j] P(j) written,
  * [248+j] Q K^T(j) issued, [368+j] P V(j) issued, each in ns after [0].
- * gattn_decode on its tensor-core path (K=V, 8 or 16 query heads per kv
- * head) writes the same header [0..5] per split CTA (CTA index
- * (b * num_kv_heads + kv_head) * splits + split), and per key tile j < 24:
- * [8+j] tile landed, [32+j] key prologue done, [56+j] Q K^T(j) issued,
- * [80+j] S(j) seen by the softmax, [104+j] P(j) written, [128+j] P V(j)
- * issued, [152+j] tile load issued, [176+j] key norms summed, [200+j]
- * tile maxima agreed, [224+j] P^T stored, [248+j] P^T slot free, [272+j]
- * P^T complete (seen by the P V issuer), [296+j] angles advanced, and
- * per-warp completion of the key prologue ([320/344/368+j], warps 5-7) and
- * of the softmax ([392/416/440+j], warps 1-3).
  * Whole prompts of head_dim-512 layers with an even number of query heads per
  * kv head run on SM pairs: there CTA i of the first bytes/4096 writes [0]
  * start, [1] SM id, [2] its rank in the pair, [3] items it takes, [4] key

@@ -208,6 +208,14 @@ DEC_CASES = [
     ("keqv_g16_d512_w512", W.Layer(num_heads=16, num_kv_heads=1, head_dim=512, window=512,
                                    rotary_fraction=0.25, scalar=512.0, k_eq_v=True),
      [100, 513, 2000]),
+    # no rotation and no norm: the key warps touch only a chunk's ragged last
+    # tile; several full chunks of 2048 keys stream through the ring
+    ("keqv_g16_d512_norope", W.Layer(num_heads=16, num_kv_heads=1, head_dim=512, rotary_fraction=0.0,
+                                     scalar=512.0, k_eq_v=True), [1, 128, 129, 2048, 4100]),
+    ("keqv_g8_d256_r64_w1000", W.Layer(num_heads=8, num_kv_heads=1, head_dim=256, rotary_fraction=0.25,
+                                       k_eq_v=True, qk_norm=W.NORM_W, window=1000), [999, 1000, 1001, 3333]),
+    ("keqv_g16_d512_r32_norm1", W.Layer(num_heads=16, num_kv_heads=1, head_dim=512, rotary_fraction=0.0625,
+                                        scalar=512.0, k_eq_v=True, qk_norm=W.NORM_ONE_PLUS_W), [257, 1999, 6000]),
 ]
 
 
