@@ -303,10 +303,10 @@ def make_chunk(wl, dev):
 
 def dominant_decode_src(L: W.Layer, int8: bool = False) -> str:
     """Source of the split kernel a decode layer runs (the step's dominant kernel): the
-    tensor-core one for K=V with 8 or 16 query heads per kv head (bf16 caches), the
-    CUDA-core one for 1, 2 or 4, else the split kernel in the prologue/combine file."""
+    tensor-core one for K=V with 8 or 16 query heads per kv head (bf16 or int8 caches),
+    the CUDA-core one for 1, 2 or 4, else the split kernel in the prologue/combine file."""
     G = L.num_heads // L.num_kv_heads
-    if L.k_eq_v and G in (8, 16) and not int8:
+    if L.k_eq_v and G in (8, 16):
         return "gemma_family_decoder_b200/csrc/decode_tc.cu"
     if G in (1, 2, 4):
         return "gemma_family_decoder_b200/csrc/decode_simt.cu"

@@ -20,11 +20,19 @@
 // the same (m, l, O) partial per (b, head, chunk) as the other split kernels,
 // merged by decode_combine_kernel.
 //
+// An int8 cache (Q8: codes c and one fp32 scale s per row, k = c * s) runs
+// the same products on the codes themselves: integers in [-127, 127] are
+// exact in bf16.  Each unit's codes land in the upper half of its slot, and
+// the key warps widen them in place to the bf16 layout of the tile; the row
+// scale then goes into the key's factor on S^T (s / sqrt(s^2 mean(c^2) + eps)
+// under QK-norm, s without) and into P^T for P V (P(key) * s(key)), the
+// softmax sums staying those of the unscaled P.
+//
 // Warps: 0-3 softmax over each tile's S^T (thread = key; TMEM lane = key) and
-// the epilogue (thread = value dim); 4-11 two threads per key: key norms, the
-// in-place rotation, and zeroing of rows past the chunk's end (so that P V
-// multiplies 0 by 0 there, not by stale or poisoned data); 12 TMA producer;
-// 13 MMA issuer.
+// the epilogue (thread = value dim); 4-11 two threads per key: int8 widening,
+// key norms, the in-place rotation, and zeroing of rows past the chunk's end
+// (so that P V multiplies 0 by 0 there, not by stale or poisoned data); 12 TMA
+// producer; 13 MMA issuer.
 #include <cuda_bf16.h>
 
 #include "gattn_internal.h"
@@ -52,8 +60,9 @@ struct DecShape {
   static constexpr int OFF_Q = OFF_RING + NSLOT * UNIT;
   static constexpr int OFF_P = OFF_Q + NBX * QSLAB;
   static constexpr int OFF_RSTEP = OFF_P + 2 * PSLAB;        // (cos, sin) of a 128-position step, [64]
-  static constexpr int OFF_RN = OFF_RSTEP + 64 * 8;          // key 1/rms, [2][128]
-  static constexpr int OFF_RED = OFF_RN + 2 * TK * 4;        // head maxima [2][4][16], sums [4][16]
+  static constexpr int OFF_RN = OFF_RSTEP + 64 * 8;          // key factor on S^T (1/rms, with int8 s/rms), [2][128]
+  static constexpr int OFF_SC = OFF_RN + 2 * TK * 4;         // int8 row scales, [2][128]
+  static constexpr int OFF_RED = OFF_SC + 2 * TK * 4;        // head maxima [2][4][16], sums [4][16]
   static constexpr int OFF_BAR = OFF_RED + 3 * 4 * 16 * 4;
   static constexpr int NBAR = 24;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -69,8 +78,13 @@ struct DecShape {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
+// An int8 unit: its codes (two boxes of 128 dims x 128 keys) land in the upper
+// half of the slot, then are widened to the four bf16 boxes in place.
+constexpr int kQ8Box = 128 * 128;
+
 struct DecTcParams {
-  CUtensorMap tm_k;   // cache [B][Lmax][Hkv][D], box 64 dims x 128 keys (keys = values)
+  CUtensorMap tm_k;   // cache [B][Lmax][Hkv][D], box 64 dims x 128 keys (keys = values);
+                      // int8 codes: box 128 dims x 128 keys
   DecodeArgs da;
   LayerArgs la;
   uint64_t timeout_ns;
@@ -111,7 +125,7 @@ __device__ __forceinline__ UnitOf unit_of(int u, int n) {
 
 }  // namespace
 
-template <int D, int G>
+template <int D, int G, bool Q8>
 __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(const __grid_constant__ DecTcParams P) {
   using C = DecShape<D, G>;
   const DecodeArgs& da = P.da;
@@ -155,6 +169,8 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);    // [3][4][16]
   float* rnbuf = reinterpret_cast<float*>(smem + C::OFF_RN);   // [2][128]
+  float* scbuf = reinterpret_cast<float*>(smem + C::OFF_SC);   // [2][128]
+  const bool key_factor = Q8 || la.qk_norm;                     // a per-key factor on S^T
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -257,10 +273,11 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
       const int slot = j & 1;
       const uint32_t par = (j >> 1) & 1;
       bool okj = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[slot], par, tmo, da.status, abort_flag));
-      float rn = 1.f;
-      if (la.qk_norm) {
+      float rn = 1.f, sk = 1.f;
+      if (key_factor) {
         okj = okj && __all_sync(0xffffffffu, mbar_wait(&rn_full[slot], par, tmo, da.status, abort_flag));
         rn = rnbuf[slot * C::TK + t];
+        if (Q8) sk = scbuf[slot * C::TK + t];
         mbar_arrive(&rn_empty[slot]);
       }
       float x[G];
@@ -325,10 +342,15 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
         const int kp = t & 62;  // even key of the pair, within the atom
 #pragma unroll
         for (int h = 0; h < G; h += 2) {
-          const float p0 = ex2(x[h] - (m[h] == -INFINITY ? 0.f : m[h]));
-          const float p1 = ex2(x[h + 1] - (m[h + 1] == -INFINITY ? 0.f : m[h + 1]));
+          float p0 = ex2(x[h] - (m[h] == -INFINITY ? 0.f : m[h]));
+          float p1 = ex2(x[h + 1] - (m[h + 1] == -INFINITY ? 0.f : m[h + 1]));
           lp[h] = lp[h] * alpha[h] + p0;
           lp[h + 1] = lp[h + 1] * alpha[h + 1] + p1;
+          if (Q8) {
+            // P V runs on the codes: the key's scale goes into its P
+            p0 *= sk;
+            p1 *= sk;
+          }
           const float recv = __shfl_xor_sync(0xffffffffu, odd ? p0 : p1, 1);
           const int hh = h + (odd ? 1 : 0);
           *reinterpret_cast<uint32_t*>(pbase + hh * 128 + (((kp >> 3) ^ (hh & 7)) << 4) + (kp & 7) * 2) =
@@ -443,6 +465,12 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
       x[4] *= g1.x + koff; x[5] *= g1.y + koff; x[6] *= g1.z + koff; x[7] *= g1.w + koff;
     };
     float ss = 0.f;
+    // int8: the row scale of this thread's key in the current tile and the next
+    float s_cur = 0.f, s_next = 0.f;
+    auto load_scale = [&](int tile) -> float {
+      const int key = start + tile * C::TK + k;
+      return key < end ? __ldg(da.ks + (static_cast<size_t>(b) * da.max_len + key) * la.Hkv + kvh) : 0.f;
+    };
     // the 256 threads leave the loop together, at a unit's first barrier, or
     // not at all (a failed wait is carried to the next unit in `okc`)
     bool okc = true;
@@ -455,6 +483,44 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
       uint8_t* ub = smem + C::OFF_RING + slot * C::UNIT;
       const int key0 = start + uo.tile * C::TK;
       const int nvalid = min(C::TK, end - key0);
+      if constexpr (Q8) {
+        // Widen the unit's codes (the slot's upper half: code box 0 = the
+        // unit's dims 0-127, box 1 = dims 128-255; 128 B per key, 128-byte
+        // swizzle) to the four bf16 boxes.  Box 0 goes to bf16 boxes 0-1 (the
+        // lower half); box 1 is read by every thread before any of it is
+        // overwritten by bf16 boxes 2-3.
+        const uint8_t* q8 = ub + C::UNIT / 2;
+        auto widen = [&](const uint4 w, int cb) {  // 16 codes -> bf16 chunks cb, cb + 1
+          float2 a[8];
+          unpack_i8x4(w.x, a[0], a[1]);
+          unpack_i8x4(w.y, a[2], a[3]);
+          unpack_i8x4(w.z, a[4], a[5]);
+          unpack_i8x4(w.w, a[6], a[7]);
+          *tile_chunk(ub, C::BOX, k, cb) = make_uint4(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y),
+                                                      pack_bf16x2(a[2].x, a[2].y), pack_bf16x2(a[3].x, a[3].y));
+          *tile_chunk(ub, C::BOX, k, cb + 1) = make_uint4(pack_bf16x2(a[4].x, a[4].y), pack_bf16x2(a[5].x, a[5].y),
+                                                          pack_bf16x2(a[6].x, a[6].y), pack_bf16x2(a[7].x, a[7].y));
+        };
+        uint4 w1[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int i = hf + 2 * m;  // 16-code chunk of the box
+          const int off = k * 128 + ((i ^ (k & 7)) << 4);
+          const uint4 w0 = *reinterpret_cast<const uint4*>(q8 + off);
+          w1[m] = *reinterpret_cast<const uint4*>(q8 + kQ8Box + off);
+          widen(w0, 2 * i);
+        }
+        named_barrier(2, 256);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) widen(w1[m], 16 + 2 * (hf + 2 * m));
+        named_barrier(2, 256);
+        if (!uo.pv && uo.c == 0) {
+          // this tile's row scales (loaded a tile ahead) and the next tile's
+          if (uo.tile == 0) s_next = load_scale(0);
+          s_cur = s_next;
+          s_next = uo.tile + 1 < ntiles ? load_scale(uo.tile + 1) : 0.f;
+        }
+      }
       if (!uo.pv) {
         if (la.qk_norm) {
           float acc[8];
@@ -533,15 +599,24 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
             }
           }
         }
-        if (uo.c == C::NCH - 1 && la.qk_norm) {
-          // the key's norm: both threads' sums; the softmax reads it per tile
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          const float rn = rsqrtf(ss / static_cast<float>(D) + la.eps);
+        if (uo.c == C::NCH - 1 && key_factor) {
+          // the key's factor on S^T, read by the softmax per tile: 1/rms(k)
+          // from both threads' sums; with int8 codes k = c s, so the factor is
+          // s / sqrt(s^2 mean(c^2) + eps), or s without QK-norm
+          float f = s_cur;
+          if (la.qk_norm) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            const float ms = ss / static_cast<float>(D);
+            f = Q8 ? s_cur * rsqrtf(s_cur * s_cur * ms + la.eps) : rsqrtf(ms + la.eps);
+          }
           ss = 0.f;
           const int ts = uo.tile & 1;
           okc = __all_sync(0xffffffffu, mbar_wait(&rn_empty[ts], ((uo.tile >> 1) & 1) ^ 1, tmo, da.status,
                                                   abort_flag));
-          if (okc && hf == 0) rnbuf[ts * C::TK + k] = rn;
+          if (okc && hf == 0) {
+            rnbuf[ts * C::TK + k] = f;
+            if (Q8) scbuf[ts * C::TK + k] = s_cur;
+          }
           mbar_arrive(&rn_full[ts]);
         }
       } else if (k >= nvalid) {
@@ -565,11 +640,18 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
         const int slot = u % C::NSLOT;
         if (!mbar_wait(&empty[slot], ((u / C::NSLOT) & 1) ^ 1, tmo, da.status, abort_flag)) break;
         uint8_t* ub = smem + C::OFF_RING + slot * C::UNIT;
-        mbar_arrive_expect_tx(&full[slot], C::UNIT);
+        mbar_arrive_expect_tx(&full[slot], Q8 ? C::UNIT / 2 : C::UNIT);
+        if constexpr (Q8) {
 #pragma unroll
-        for (int bx = 0; bx < C::UB; ++bx)
-          tma_load_4d(ub + bx * C::BOX, &P.tm_k, &full[slot], (uo.db * C::UB + bx) * 64, kvh,
-                      start + uo.tile * C::TK, b);
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_4d(ub + C::UNIT / 2 + bx * kQ8Box, &P.tm_k, &full[slot], uo.db * 256 + bx * 128, kvh,
+                        start + uo.tile * C::TK, b);
+        } else {
+#pragma unroll
+          for (int bx = 0; bx < C::UB; ++bx)
+            tma_load_4d(ub + bx * C::BOX, &P.tm_k, &full[slot], (uo.db * C::UB + bx) * 64, kvh,
+                        start + uo.tile * C::TK, b);
+        }
         issued = u + 1;
       }
       // let every issued copy land before the CTA can exit
@@ -648,16 +730,17 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool Q8>
 static cudaError_t run_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
   using C = DecShape<D, G>;
   DecTcParams P;
-  if (!encode_tmap_bshd(&P.tm_k, da.k, da.B, da.max_len, la.Hkv, D, C::TK))
-    return cudaErrorInvalidValue;
+  const bool enc = Q8 ? encode_tmap_bshd_u8(&P.tm_k, da.kq, da.B, da.max_len, la.Hkv, D, 128, C::TK)
+                      : encode_tmap_bshd(&P.tm_k, da.k, da.B, da.max_len, la.Hkv, D, C::TK);
+  if (!enc) return cudaErrorInvalidValue;
   P.da = da;
   P.la = la;
   P.timeout_ns = wait_timeout_ns();
-  auto kern = decode_tc_kernel<D, G>;
+  auto kern = decode_tc_kernel<D, G, Q8>;
   constexpr int kMaxDev = 64;
   static bool attr_set[kMaxDev] = {};
   int dev = 0;
@@ -679,8 +762,14 @@ bool decode_tc_supported(const LayerArgs& la) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
-  if (la.D == 512) return la.G == 16 ? run_decode_tc<512, 16>(da, la, s) : run_decode_tc<512, 8>(da, la, s);
-  return la.G == 16 ? run_decode_tc<256, 16>(da, la, s) : run_decode_tc<256, 8>(da, la, s);
+  if (da.kq) {
+    if (la.D == 512)
+      return la.G == 16 ? run_decode_tc<512, 16, true>(da, la, s) : run_decode_tc<512, 8, true>(da, la, s);
+    return la.G == 16 ? run_decode_tc<256, 16, true>(da, la, s) : run_decode_tc<256, 8, true>(da, la, s);
+  }
+  if (la.D == 512)
+    return la.G == 16 ? run_decode_tc<512, 16, false>(da, la, s) : run_decode_tc<512, 8, false>(da, la, s);
+  return la.G == 16 ? run_decode_tc<256, 16, false>(da, la, s) : run_decode_tc<256, 8, false>(da, la, s);
 }
 
 }  // namespace gattn

@@ -86,7 +86,8 @@ void decode_plan(const LayerArgs& la, int B, int max_len, int* nsplit, int* chun
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 // Tensor-core split kernel: K=V layers with 8 or 16 query heads per kv head,
-// head_dim 256 or 512 and at most 128 rotated dims (same partial format).
+// head_dim 256 or 512 and at most 128 rotated dims, bf16 or int8 caches (same
+// partial format).
 bool decode_tc_supported(const LayerArgs& la);
 cudaError_t launch_decode_tc(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s);
 // Persistent CUDA-core split kernel for 1, 2 or 4 query heads per kv head
@@ -158,5 +159,8 @@ uint64_t wait_timeout_ns();
 // TMA descriptor encoding through the driver entry point (no -lcuda needed).
 bool encode_tmap_bshd(CUtensorMap* map, const void* base, int B, int S, int Hkv, int D,
                       int box_rows);
+// The same view of an int8 cache [B][S][Hkv][D] (codes), box box_inner bytes x box_rows rows.
+bool encode_tmap_bshd_u8(CUtensorMap* map, const void* base, int B, int S, int Hkv, int D, int box_inner,
+                         int box_rows);
 
 }  // namespace gattn

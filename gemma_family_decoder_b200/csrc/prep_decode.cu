@@ -494,8 +494,9 @@ static cudaError_t run_decode_split(const DecodeArgs& da, const LayerArgs& la, c
 }
 
 cudaError_t launch_decode_split(const DecodeArgs& da, const LayerArgs& la, cudaStream_t s) {
-  // an int8 cache (da.kq): the persistent CUDA-core kernel, else the split kernel below
-  if (!da.kq && decode_tc_supported(la)) return launch_decode_tc(da, la, s);
+  // bf16 or int8 caches: the tensor-core kernel (K=V, 8 or 16 query heads per kv head),
+  // the persistent CUDA-core kernel (1, 2 or 4), else the split kernel below
+  if (decode_tc_supported(la)) return launch_decode_tc(da, la, s);
   if (decode_simt_supported(la)) return launch_decode_simt(da, la, s);
   const int hpw = la.G <= 2 ? la.G : la.G / 4;
   if (la.D == 256) {

@@ -269,9 +269,11 @@ int gattn_kv_quantize(const gattn_bf16* x, int8_t* codes, float* scales, int64_t
  * Every other argument, the workspace size (gattn_decode_workspace_size) and
  * the errors are those of gattn_decode, and so are the layers it takes: 1, 2 or
  * 4 query heads per kv head (head_dim 512: 1 or 2, and 1, 2, 4 or 8 kv heads)
- * run the persistent CUDA-core split kernel; the rest (8 or 16 query heads per
- * kv head, the Gemma 4 K=V global layer among them) a slower CUDA-core split
- * kernel that dequantises row by row (the tensor-core decode reads bf16 only). */
+ * run the persistent CUDA-core split kernel; K=V layers with 8 or 16 query
+ * heads per kv head (the Gemma 4 global layer) the tensor-core kernel, whose
+ * MMAs take the codes themselves (integers, exact in bf16) and apply each row's
+ * scale to its logits and its softmax weights; the rest a slower CUDA-core split
+ * kernel that dequantises row by row. */
 int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k_scales,
                       const int8_t* v_codes_or_null, const float* v_scales_or_null, const int32_t* seq_lens,
                       gattn_bf16* out, int32_t batch, int32_t max_len, const gattn_cfg* cfg, void* workspace,

@@ -1,5 +1,6 @@
 """GPU parity of the int8 KV cache: gattn_kv_quantize and gattn_decode_int8 (the persistent
-CUDA-core kernel for 1, 2 or 4 query heads per kv head, the split kernel for 8 or 16).
+CUDA-core kernel for 1, 2 or 4 query heads per kv head, the tensor-core kernel for K=V
+layers with 8 or 16, the split kernel for the rest).
 
 The quantiser is integer work decided by float32 division on both sides, so
 its codes and scales must equal the oracle's bit for bit.  The int8 decode is
@@ -115,10 +116,18 @@ INT8_CASES = [
                                          k_eq_v=True), [1, 9, 64, 65]),
     ("g2_d256_r16_cap_w5", W.Layer(num_heads=8, num_kv_heads=4, head_dim=256, rotary_fraction=0.0625,
                                    softcap=30.0, window=5), [1, 4, 5, 6, 40]),
-    # 8 or 16 query heads per kv head: the CUDA-core split kernel reading int8 rows
+    # K=V with 8 or 16 query heads per kv head: the tensor-core kernel on the codes
     ("global_keqv_g16_d512", W.GEMMA4_DECODE_GLOBAL.layer, [1, 700, 2049, 2500]),
     ("keqv_g8_d512_norm", W.Layer(num_heads=8, num_kv_heads=1, head_dim=512, rope_theta=1e6, rotary_fraction=0.25,
                                   scalar=512.0, k_eq_v=True, qk_norm=W.NORM_W), [3, 65, 700]),
+    ("keqv_g16_d512_norope", W.Layer(num_heads=16, num_kv_heads=1, head_dim=512, rotary_fraction=0.0,
+                                     scalar=512.0, k_eq_v=True), [1, 128, 129, 2048, 4100]),
+    ("keqv_g16_d256_cap_r16_norm1", W.Layer(num_heads=32, num_kv_heads=2, head_dim=256, rotary_fraction=0.0625,
+                                            softcap=30.0, k_eq_v=True, qk_norm=W.NORM_ONE_PLUS_W, window=200),
+     [1, 150, 199, 200, 201, 1300]),
+    ("keqv_g8_d256_r64_w1000_norm", W.Layer(num_heads=8, num_kv_heads=1, head_dim=256, rotary_fraction=0.25,
+                                            k_eq_v=True, qk_norm=W.NORM_W, window=1000), [999, 1000, 1001, 3333]),
+    # 8 or 16 query heads per kv head without K=V: the CUDA-core split kernel
     ("g8_d256_window_cap", W.Layer(num_heads=16, num_kv_heads=2, head_dim=256, window=200, softcap=30.0),
      [1, 199, 200, 201, 900]),
 ]
@@ -144,6 +153,49 @@ def test_decode_int8_workload_matches_oracle():
     out, st = run_decode_int8(wl.layer, dq["q"], dev, seq_lens, dq["w_q"], dq["w_k"])
     assert st == 0
     assert_close(out, oracle_int8(dq, host, seq_lens, wl.layer), wl.name + " int8")
+
+
+@pytest.mark.parametrize("wl", [W.GEMMA4_DECODE_GLOBAL, W.GEMMA4_DECODE_GLOBAL_NORM], ids=lambda w: w.name)
+def test_decode_int8_global_workload_matches_oracle(wl):
+    # the Gemma 4 global K=V layer over a full-size int8 cache (the tensor-core kernel), every
+    # fourth batch row against the oracle
+    dq = W.decode_inputs(wl)
+    seq_lens = dq["seq_lens"]
+    k, v, oa = decode_full_cache(wl, seq_lens)
+    kq, ks = quantize_dev(torch.nan_to_num(k))
+    del k, v
+    batches = list(range(0, wl.batch, 4))
+    kc = [None] * wl.batch
+    ksc = [None] * wl.batch
+    for b in batches:
+        L = int(seq_lens[b])
+        kc[b], ksc[b] = O.kv_quantize(oa["k_cache"][b].float().numpy())
+        assert np.array_equal(kq[b, :L].cpu().numpy(), kc[b])
+        ks[b, L:] = float("nan")
+    out, st = run_decode_int8(wl.layer, dq["q"], (kq, ks, None, None), seq_lens, dq["w_q"], dq["w_k"])
+    assert st == 0
+    ref = O.attention_decode_int8(dq["q"], kc, ksc, None, None, seq_lens, wl.layer, w_q=dq["w_q"], w_k=dq["w_k"],
+                                  batches=batches)
+    assert_close(out[batches], ref, wl.name + " int8")
+
+
+def test_decode_int8_tensor_core_zero_rows():
+    # zero rows (scale 0, codes 0) in a K=V layer on the tensor-core kernel: ordinary keys
+    # with logit 0 and value 0, under QK-norm (their norm is sqrt(eps))
+    layer = W.GEMMA4_DECODE_GLOBAL_NORM.layer
+    wl = W.DecodeWorkload("z16", layer, 2, 1, 700, seed=29, gain_mean=1.0, gain_std=0.1)
+    dq = W.decode_inputs(wl)
+    seq_lens = torch.tensor([700, 333], dtype=torch.int32)
+    k, v, oa = decode_full_cache(wl, seq_lens, max_len=700)
+    k = torch.nan_to_num(k)
+    k[0, 10:20] = 0.0
+    k[1, 128:300] = 0.0
+    kq, ks = quantize_dev(k)
+    out, st = run_decode_int8(layer, dq["q"], (kq, ks, None, None), seq_lens, dq["w_q"], dq["w_k"])
+    assert st == 0
+    kd = [O.kv_dequantize(*O.kv_quantize(k[b, :int(seq_lens[b])].float().cpu().numpy())) for b in range(2)]
+    ref = O.attention_decode(dq["q"], kd, None, seq_lens, layer, w_q=dq["w_q"], w_k=dq["w_k"])
+    assert_close(out, ref, "zero rows, tensor core")
 
 
 def test_decode_int8_zero_rows_and_bad_length():
