@@ -191,86 +191,10 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
   return u;
 }
 
-// Query prologue of a prefill tile held in shared memory (128 rows, 128-byte
-// swizzled 64-dim slabs), in place, on one row: RMSNorm over the row, then RoPE
-// with angles computed here (pair t turns theta^(-2t/F) / 2pi per position,
-// built as a geometric sequence in double precision), so the only global read
-// is the row's position.  A row may be split between threads: tile_row_sumsq
-// gives the partial sum of squares of chunks [c_lo, c_hi), and
-// tile_row_prologue rotates the pair chunks [pc_lo, pc_hi) (chunk c with chunk
-// c + R/16) and scales the unrotated chunks [uc_lo, uc_hi) by the norm.
+// 16-byte chunk c (8 dims) of row r of a tile held in shared memory as
+// 128-byte swizzled 64-dim slabs of slab_bytes each (the TMA layout).
 __device__ __forceinline__ uint4* tile_chunk(uint8_t* tile, int slab_bytes, int r, int c) {
   return reinterpret_cast<uint4*>(tile + (c >> 3) * slab_bytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ float tile_row_sumsq(uint8_t* tile, int slab_bytes, int r, int c_lo,
-                                                int c_hi) {
-  float ss = 0.f;
-#pragma unroll 4
-  for (int c = c_lo; c < c_hi; ++c) {
-    float x[8];
-    unpack8(*tile_chunk(tile, slab_bytes, r, c), x);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
-  }
-  return ss;
-}
-
-// rn: 1/rms of the whole row (ignored without QK-norm).
-__device__ __forceinline__ void tile_row_prologue(uint8_t* tile, int slab_bytes, int r, int pos,
-                                                  const LayerArgs& la, float rn, int pc_lo,
-                                                  int pc_hi, int uc_lo, int uc_hi) {
-  const float off = la.qk_norm == 1 ? 1.f : 0.f;
-  const float4* g4 = reinterpret_cast<const float4*>(la.q_norm_w);
-  auto gain8 = [&](int c, float (&x)[8]) {
-    if (!la.qk_norm) return;
-    const float4 g0 = __ldg(g4 + 2 * c), g1 = __ldg(g4 + 2 * c + 1);
-    x[0] *= rn * (g0.x + off); x[1] *= rn * (g0.y + off);
-    x[2] *= rn * (g0.z + off); x[3] *= rn * (g0.w + off);
-    x[4] *= rn * (g1.x + off); x[5] *= rn * (g1.y + off);
-    x[6] *= rn * (g1.z + off); x[7] *= rn * (g1.w + off);
-  };
-  const int h8 = la.rot >> 4;  // 8-dim chunks in half the rotated slice
-  if (la.rot > 0 && pc_lo < pc_hi) {
-    const double q = la.rope_ratio;
-    double qp[8];  // q^e, e < 8
-    qp[0] = 1.0;
-#pragma unroll
-    for (int e = 1; e < 8; ++e) qp[e] = qp[e - 1] * q;
-    const double q8 = qp[7] * q;
-    double f8 = 0.15915494309189533576888376337251;  // turns per radian: pair 0
-    for (int c = 0; c < pc_lo; ++c) f8 *= q8;
-#pragma unroll 2
-    for (int c = pc_lo; c < pc_hi; ++c) {
-      uint4* cx = tile_chunk(tile, slab_bytes, r, c);
-      uint4* cy = tile_chunk(tile, slab_bytes, r, c + h8);
-      float x[8], y[8];
-      unpack8(*cx, x);
-      unpack8(*cy, y);
-      gain8(c, x);
-      gain8(c + h8, y);
-      float xo[8], yo[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float2 cs = rope_cos_sin(pos, f8 * qp[e]);
-        xo[e] = x[e] * cs.x - y[e] * cs.y;
-        yo[e] = y[e] * cs.x + x[e] * cs.y;
-      }
-      *cx = pack8(xo);
-      *cy = pack8(yo);
-      f8 *= q8;
-    }
-  }
-  if (la.qk_norm) {
-#pragma unroll 4
-    for (int c = uc_lo; c < uc_hi; ++c) {
-      uint4* cx = tile_chunk(tile, slab_bytes, r, c);
-      float x[8];
-      unpack8(*cx, x);
-      gain8(c, x);
-      *cx = pack8(x);
-    }
-  }
 }
 
 }  // namespace gattn
