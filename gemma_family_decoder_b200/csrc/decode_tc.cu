@@ -483,6 +483,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
       uint8_t* ub = smem + C::OFF_RING + slot * C::UNIT;
       const int key0 = start + uo.tile * C::TK;
       const int nvalid = min(C::TK, end - key0);
+      bool arrived = false;  // this unit already announced ready
       if constexpr (Q8) {
         // Widen the unit's codes (the slot's upper half: code box 0 = the
         // unit's dims 0-127, box 1 = dims 128-255; 128 B per key, 128-byte
@@ -580,6 +581,11 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
               *tile_chunk(ub, C::BOX, k, c + h8) = make_uint4(yo[0], yo[1], yo[2], yo[3]);
             }
           }
+          // the unit is ready for its MMAs now; the angles of the next tile
+          // are advanced after (nothing waits for them until then)
+          fence_proxy_async_smem();
+          mbar_arrive(&ready[slot]);
+          arrived = true;
           if (((uo.tile + 1) & 31) != 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -624,8 +630,10 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
 #pragma unroll 4
         for (int c = hf; c < 4 * 8; c += 2) *tile_chunk(ub, C::BOX, k, c) = z;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&ready[slot]);
+      if (!arrived) {
+        fence_proxy_async_smem();
+        mbar_arrive(&ready[slot]);
+      }
     }
   }
   else if (warp == 12) {
