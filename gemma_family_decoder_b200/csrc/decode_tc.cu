@@ -22,8 +22,9 @@
 //
 // An int8 cache (Q8: codes c and one fp32 scale s per row, k = c * s) runs
 // the same products on the codes themselves: integers in [-127, 127] are
-// exact in bf16.  Each unit's codes land in the upper half of its slot, and
-// the key warps widen them in place to the bf16 layout of the tile; the row
+// exact in fp16, which that instance's MMAs take (Q and P in fp16 as well).
+// Each unit's codes land in the upper half of its slot, and the key warps
+// widen them in place to the fp16 layout of the tile; the row
 // scale then goes into the key's factor on S^T (s / sqrt(s^2 mean(c^2) + eps)
 // under QK-norm, s without) and into P^T for P V (P(key) * s(key)), the
 // softmax sums staying those of the unscaled P.
@@ -34,6 +35,7 @@
 // (so that P V multiplies 0 by 0 there, not by stale or poisoned data); 12 TMA
 // producer; 13 MMA issuer.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "gattn_internal.h"
 #include "kernels/common.cuh"
@@ -91,6 +93,42 @@ struct DecTcParams {
 };
 
 constexpr float kLog2eD = 1.4426950408889634f;
+
+// The MMA operands' element type: bf16 over a bf16 cache; fp16 over an int8
+// cache (H), whose codes widen to fp16 in two operations per pair (below), Q
+// and P then fp16 too (a kind::f16 MMA takes one type for A and B).
+template <bool H>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (H) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    return pack_bf16x2(lo, hi);
+  }
+}
+template <bool H>
+__device__ __forceinline__ void unpack8x(const uint4 u, float (&x)[8]) {
+  if constexpr (H) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+  } else {
+    unpack8(u, x);
+  }
+}
+template <bool H>
+__device__ __forceinline__ uint4 pack8x(const float (&x)[8]) {
+  return make_uint4(pack2<H>(x[0], x[1]), pack2<H>(x[2], x[3]), pack2<H>(x[4], x[5]), pack2<H>(x[6], x[7]));
+}
+// Instruction descriptor of kind::f16 with fp16 A and B (the format fields of
+// the bf16 descriptor cleared), fp32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, a_mn_major, b_mn_major) & ~((7u << 7) | (7u << 10));
+}
 
 // Ring unit u of a chunk of n tiles: unit blocks in the order Q K^T(0),
 // Q K^T(1), P V(0), Q K^T(2), P V(1), ..., Q K^T(n-1), P V(n-2), P V(n-1),
@@ -231,7 +269,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           x[hh][i][6] *= g1.z + koff; x[hh][i][7] *= g1.w + koff;
         }
         *reinterpret_cast<uint4*>(smem + C::OFF_Q + (c >> 3) * C::QSLAB + h * 128 +
-                                  (((c & 7) ^ (h & 7)) << 4)) = pack8(x[hh][i]);
+                                  (((c & 7) ^ (h & 7)) << 4)) = pack8x<Q8>(x[hh][i]);
       }
     }
     if constexpr (G < C::NQ) {
@@ -354,7 +392,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           const float recv = __shfl_xor_sync(0xffffffffu, odd ? p0 : p1, 1);
           const int hh = h + (odd ? 1 : 0);
           *reinterpret_cast<uint32_t*>(pbase + hh * 128 + (((kp >> 3) ^ (hh & 7)) << 4) + (kp & 7) * 2) =
-              odd ? pack_bf16x2(recv, p1) : pack_bf16x2(p0, recv);
+              odd ? pack2<Q8>(recv, p1) : pack2<Q8>(p0, recv);
         }
       }
       // O must hold P V of every earlier tile before it is rescaled; seeing
@@ -487,20 +525,28 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
       if constexpr (Q8) {
         // Widen the unit's codes (the slot's upper half: code box 0 = the
         // unit's dims 0-127, box 1 = dims 128-255; 128 B per key, 128-byte
-        // swizzle) to the four bf16 boxes.  Box 0 goes to bf16 boxes 0-1 (the
+        // swizzle) to the four fp16 boxes.  Box 0 goes to fp16 boxes 0-1 (the
         // lower half); box 1 is read by every thread before any of it is
-        // overwritten by bf16 boxes 2-3.
+        // overwritten by fp16 boxes 2-3.  A code c widens exactly: the fp16 of
+        // bits 0x6400 | (c + 128) is 1024 + c + 128 (fp16 steps by 1 in
+        // [1024, 2048)), so one byte permute places two codes under that
+        // exponent byte and one packed subtract of 1152 leaves c.
         const uint8_t* q8 = ub + C::UNIT / 2;
-        auto widen = [&](const uint4 w, int cb) {  // 16 codes -> bf16 chunks cb, cb + 1
-          float2 a[8];
-          unpack_i8x4(w.x, a[0], a[1]);
-          unpack_i8x4(w.y, a[2], a[3]);
-          unpack_i8x4(w.z, a[4], a[5]);
-          unpack_i8x4(w.w, a[6], a[7]);
-          *tile_chunk(ub, C::BOX, k, cb) = make_uint4(pack_bf16x2(a[0].x, a[0].y), pack_bf16x2(a[1].x, a[1].y),
-                                                      pack_bf16x2(a[2].x, a[2].y), pack_bf16x2(a[3].x, a[3].y));
-          *tile_chunk(ub, C::BOX, k, cb + 1) = make_uint4(pack_bf16x2(a[4].x, a[4].y), pack_bf16x2(a[5].x, a[5].y),
-                                                          pack_bf16x2(a[6].x, a[6].y), pack_bf16x2(a[7].x, a[7].y));
+        const __half2 k1152 = __floats2half2_rn(1152.f, 1152.f);
+        auto widen = [&](const uint4 w, int cb) {  // 16 codes -> fp16 chunks cb, cb + 1
+          const uint32_t ws[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u, w.w ^ 0x80808080u};
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            // codes 4q, 4q+1 and 4q+2, 4q+3 as (low, high) halves
+            uint32_t lo = __byte_perm(ws[q], 0x64646464u, 0x4140), hi = __byte_perm(ws[q], 0x64646464u, 0x4342);
+            __half2 vl = __hsub2(*reinterpret_cast<__half2*>(&lo), k1152);
+            __half2 vh = __hsub2(*reinterpret_cast<__half2*>(&hi), k1152);
+            h[2 * q] = *reinterpret_cast<uint32_t*>(&vl);
+            h[2 * q + 1] = *reinterpret_cast<uint32_t*>(&vh);
+          }
+          *tile_chunk(ub, C::BOX, k, cb) = make_uint4(h[0], h[1], h[2], h[3]);
+          *tile_chunk(ub, C::BOX, k, cb + 1) = make_uint4(h[4], h[5], h[6], h[7]);
         };
         uint4 w1[4];
 #pragma unroll
@@ -530,7 +576,7 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
 #pragma unroll 4
           for (int c = hf; c < 4 * 8; c += 2) {
             float xx[8];
-            unpack8(*tile_chunk(ub, C::BOX, k, c), xx);
+            unpack8x<Q8>(*tile_chunk(ub, C::BOX, k, c), xx);
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
               const float2 v = make_float2(xx[e], xx[e + 1]);
@@ -560,8 +606,8 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
           for (int i = 0; i < 4; ++i) {
             const int c = hf + 2 * i;
             float x[8], y[8];
-            unpack8(ux[i], x);
-            unpack8(uy[i], y);
+            unpack8x<Q8>(ux[i], x);
+            unpack8x<Q8>(uy[i], y);
             gain8(c, x);
             gain8(c + h8, y);
             // two pairs per packed fp32x2 instruction
@@ -573,8 +619,8 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
               const float2 x2 = make_float2(x[e], x[e + 1]), y2 = make_float2(y[e], y[e + 1]);
               const float2 a = __ffma2_rn(x2, co, __fmul2_rn(y2, make_float2(-si.x, -si.y)));
               const float2 bb = __ffma2_rn(y2, co, __fmul2_rn(x2, si));
-              xo[e >> 1] = pack_bf16x2(a.x, a.y);
-              yo[e >> 1] = pack_bf16x2(bb.x, bb.y);
+              xo[e >> 1] = pack2<Q8>(a.x, a.y);
+              yo[e >> 1] = pack2<Q8>(bb.x, bb.y);
             }
             if (c < h8) {
               *tile_chunk(ub, C::BOX, k, c) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
@@ -675,8 +721,8 @@ __global__ void __launch_bounds__(DecShape<D, G>::THREADS, 1) decode_tc_kernel(c
     // O^T += V^T . P^T (A = two value boxes, MN-major, M=128 dims; B = P^T,
     // K-major, N=16); the first unit of tile j waits for P^T(j).
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::NQ, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::NQ, true, false);
+      constexpr uint32_t idesc_qk = Q8 ? idesc_f16_f32(128, C::NQ, false, false) : idesc_bf16_f32(128, C::NQ, false, false);
+      constexpr uint32_t idesc_pv = Q8 ? idesc_f16_f32(128, C::NQ, true, false) : idesc_bf16_f32(128, C::NQ, true, false);
       bool ok = mbar_wait(q_ready, 0, tmo, da.status, abort_flag);
       for (int u = 0; u < nunits && ok; ++u) {
         const UnitOf uo = unit_of<C::NCH>(u, ntiles);
