@@ -271,7 +271,7 @@ int gattn_kv_quantize(const gattn_bf16* x, int8_t* codes, float* scales, int64_t
  * 4 query heads per kv head (head_dim 512: 1 or 2, and 1, 2, 4 or 8 kv heads)
  * run the persistent CUDA-core split kernel; K=V layers with 8 or 16 query
  * heads per kv head (the Gemma 4 global layer) the tensor-core kernel, whose
- * MMAs take the codes themselves (integers, exact in bf16) and apply each row's
+ * MMAs take the codes themselves (integers, exact in fp16) and apply each row's
  * scale to its logits and its softmax weights; the rest a slower CUDA-core split
  * kernel that dequantises row by row. */
 int gattn_decode_int8(const gattn_bf16* q, const int8_t* k_codes, const float* k_scales,
