@@ -174,7 +174,7 @@ GEMMA3_GLOBAL_CHUNK = ChunkWorkload(
     "gemma3_1b_global_b8_chunk1024_prefix7168",
     Layer(window=0, rope_theta=1e6, **_G3), batch=8, prefix=7168, chunk=1024, seed=6)
 
-# the global K=V decode over an int8 cache (the CUDA-core split kernel)
+# the global K=V decode over an int8 cache (the tensor-core decode, on the codes)
 GEMMA4_DECODE_GLOBAL_INT8 = dataclasses.replace(GEMMA4_DECODE_GLOBAL, name="gemma4_12b_decode_global_keqv_int8_b64",
                                                 kv_int8=True)
 # the same decode and chunk steps over caches holding transformed keys
